@@ -1,0 +1,75 @@
+"""The oracle's pins must catch plausible mistakes (CPU only).
+
+Each case compiles a copy of oracle/ssd_oracle.c with one planted mistake (a dropped
+term, a wrong sign or index, a transposed operand) into a temporary directory and runs
+the pin tests against it: at least one pin must fail. Nothing here touches a GPU.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ssd_oracle.c")
+
+MUTANTS = {
+    "dropped D skip": ("yp[t * gw + (int64_t)i * P + p] = yv + Dh * xt[p];",
+                       "yp[t * gw + (int64_t)i * P + p] = yv;"),
+    "A sign flipped": ("const double decay = exp(dlt * Ah);", "const double decay = exp(-dlt * Ah);"),
+    "B and C exchanged": ("hp[n] = decay * hp[n] + dlt * xt[p] * Bt[n];\n                    yv += hp[n] * Ct[n];",
+                          "hp[n] = decay * hp[n] + dlt * xt[p] * Ct[n];\n                    yv += hp[n] * Bt[n];"),
+    "readout before update": ("hp[n] = decay * hp[n] + dlt * xt[p] * Bt[n];\n                    yv += hp[n] * Ct[n];",
+                              "yv += hp[n] * Ct[n];\n                    hp[n] = decay * hp[n] + dlt * xt[p] * Bt[n];"),
+    "input not scaled by delta": ("dlt * xt[p] * Bt[n]", "xt[p] * Bt[n]"),
+    "conv taps reversed": ("v += w[k] * s[t + k];", "v += w[K - 1 - k] * s[t + k];"),
+    "conv bias dropped": ("double v = bias;", "double v = 0.0;"),
+    "final conv state off by one": ("fin[k] = s[L + k];", "fin[k] = s[L + k - 1];"),
+    "gate without SiLU": ("yp[t * gw + c] * silu(zt[c]);", "yp[t * gw + c] * zt[c];"),
+    "norm by sum, not mean": ("sqrt(ss / (double)gw + d->eps)", "sqrt(ss + d->eps)"),
+    "norm weight dropped": ("yt[c] = yt[c] * inv * j->norm_w[xc0 + c];", "yt[c] = yt[c] * inv;"),
+    "softplus without log1p": ("log1p(exp(-fabs(u)))", "exp(-fabs(u))"),
+    "dt bias dropped": ("softplus(j->dt[(b * L + t) * H + h] + j->dt_bias[h])",
+                        "softplus(j->dt[(b * L + t) * H + h])"),
+    "heads strided over groups": ("const int h = g * r + i;\n            dl[t * r + i]",
+                                  "const int h = i * G + g;\n            dl[t * r + i]"),
+    "initial state ignored": ("if (j->init_ssm) memcpy(hs", "if (0) memcpy(hs"),
+}
+
+PINS = [
+    pins.test_softplus_closed_forms, pins.test_silu_closed_forms, pins.test_conv_hand_cases,
+    pins.test_recurrence_closed_form_constant_inputs, pins.test_brute_force_by_hand_L3,
+    lambda: pins.test_sequential_matches_chunked_form(8),
+    pins.test_sequential_matches_quadratic_form, pins.test_zero_step_leaves_state_and_gives_readout,
+    lambda: pins.test_split_and_chain_equals_one_call(2), pins.test_causality,
+    pins.test_gated_norm_single_channel_groups, pins.test_gated_norm_two_channel_group_by_hand,
+    pins.test_constant_gate_gives_sign_times_weight, pins.test_head_to_group_map_is_contiguous,
+    pins.test_prefill_equals_prefill_then_decode_steps,
+]
+
+
+def test_unmutated_source_passes_every_pin():
+    for pin in PINS:
+        pin()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site not found: {name}"
+    mutated = tmp_path / "mut.c"
+    mutated.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-o", str(so), str(mutated),
+                    "-lm", "-lpthread"], check=True)
+    failures = 0
+    with oracle.use_library(str(so)):
+        for pin in PINS:
+            try:
+                pin()
+            except (AssertionError, ValueError, FloatingPointError, RuntimeError):
+                failures += 1
+    assert failures >= 1, f"no pin caught the planted mistake: {name}"
