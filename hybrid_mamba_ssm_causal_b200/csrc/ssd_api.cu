@@ -1,0 +1,200 @@
+// ssd_api.cu -- the C ABI of include/ssd_mixer.h: argument checks, workspace carving
+// and kernel dispatch. No allocation, no host synchronisation (except the explicit
+// status read), no state kept between calls.
+#include <string.h>
+
+#include "../../include/ssd_mixer.h"
+#include "ssd_internal.h"
+
+namespace ssd {
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
+                                         int act)
+{
+    WorkspaceLayout w{};
+    const size_t es = act == SSD_BF16 ? 2 : 4;
+    const int64_t HP = (int64_t)H * P, Cc = HP + 2 * (int64_t)G * N;
+    const int64_t nc = Q > 0 ? (L + Q - 1) / Q : 0;
+    size_t off = 0;
+    w.status = off; off = align256(off + 256);
+    w.xbc = off;    off = align256(off + (size_t)(b * L * Cc) * es);
+    w.delta = off;  off = align256(off + (size_t)(b * H * L) * 4);
+    w.lam = off;    off = align256(off + (size_t)(b * H * L) * 4);
+    w.states = off; off = align256(off + (size_t)(b * nc * H) * (size_t)P * N * 4);
+    w.ypre = off;   off = align256(off + (size_t)(b * L * HP) * 4);
+    w.total = off;
+    return w;
+}
+
+}  // namespace ssd
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// Shape checks common to prefill and decode. Returns SSD_OK or the error.
+ssd_status check_dims(const ssd_dims* d, bool decode)
+{
+    if (!d) return SSD_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->seqlen < 0 || d->nheads <= 0 || d->headdim <= 0 || d->ngroups <= 0 ||
+        d->dstate <= 0 || !(d->eps > 0.0f))
+        return SSD_ERR_INVALID_ARG;
+    if (d->act != SSD_F32 && d->act != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    if (d->nheads % d->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (d->dconv != 4) return SSD_ERR_UNSUPPORTED;
+    if (!pow2_in(d->headdim, 16, 128) || !pow2_in(d->dstate, 16, 128)) return SSD_ERR_UNSUPPORTED;
+    if (d->nheads > 65535 || d->batch > 65535) return SSD_ERR_UNSUPPORTED;
+    if (decode) {
+        if (d->seqlen != 1) return SSD_ERR_INVALID_ARG;
+        if (!ssd::decode_supported(d->headdim, d->dstate)) return SSD_ERR_UNSUPPORTED;
+        // the group's channels and vectors live in shared memory
+        const int64_t r = d->nheads / d->ngroups;
+        if ((2 * r * d->headdim + 2 * d->dstate + r + 8) * 4 > 200 * 1024) return SSD_ERR_UNSUPPORTED;
+    } else {
+        if (d->chunk < 16 || d->chunk > 256 || d->chunk % 16 != 0) return SSD_ERR_UNSUPPORTED;
+        if (!ssd::prefill_simt_supported(d->headdim, d->dstate)) return SSD_ERR_UNSUPPORTED;
+        const int64_t nc = (d->seqlen + d->chunk - 1) / d->chunk;
+        if (nc * ((d->chunk + 63) / 64) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    }
+    return SSD_OK;
+}
+
+// Row-layout checks for one activation operand (16-byte vector access unless scalar).
+bool row_ok(const void* p, int64_t ld, int64_t width, size_t es, bool vector)
+{
+    if (!p || ld < width) return false;
+    if (vector) return aligned16(p) && ((size_t)ld * es) % 16 == 0;
+    return ((uintptr_t)p % es) == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_mixer_prefill_workspace_size(const ssd_dims* d)
+{
+    if (check_dims(d, false) != SSD_OK) return 0;
+    return ssd::prefill_workspace_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->ngroups,
+                                         d->dstate, d->chunk, d->act)
+        .total;
+}
+
+ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, const void* z,
+                             int64_t z_ld, const void* B, int64_t B_ld, const void* C, int64_t C_ld,
+                             const void* dt, int64_t dt_ld, const float* A, const float* D,
+                             const float* conv_w, const float* conv_b, const float* dt_bias,
+                             const float* norm_w, const float* init_ssm_state,
+                             const void* init_conv_state, void* y, int64_t y_ld,
+                             float* final_ssm_state, void* final_conv_state, void* workspace,
+                             size_t workspace_bytes, void* stream)
+{
+    const ssd_status ds = check_dims(d, false);
+    if (ds != SSD_OK) return ds;
+    const size_t es = d->act == SSD_BF16 ? 2 : 4;
+    const int64_t HP = (int64_t)d->nheads * d->headdim, GN = (int64_t)d->ngroups * d->dstate;
+    if (!A || !D || !conv_w || !conv_b || !dt_bias || !norm_w || !final_ssm_state || !final_conv_state)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(conv_w) || !aligned16(final_ssm_state) ||
+        (init_ssm_state && !aligned16(init_ssm_state)))
+        return SSD_ERR_UNSUPPORTED;
+    if ((init_conv_state && ((uintptr_t)init_conv_state % es)) || ((uintptr_t)final_conv_state % es))
+        return SSD_ERR_UNSUPPORTED;
+    const ssd::WorkspaceLayout wl = ssd::prefill_workspace_layout(
+        d->batch, d->seqlen, d->nheads, d->headdim, d->ngroups, d->dstate, d->chunk, d->act);
+    if (!workspace || workspace_bytes < wl.total || ((uintptr_t)workspace & 255u))
+        return SSD_ERR_INVALID_ARG;
+    if (d->seqlen > 0 && d->batch > 0) {
+        if (!x || !z || !B || !C || !dt || !y) return SSD_ERR_INVALID_ARG;
+        if (!row_ok(x, x_ld, HP, es, true) || !row_ok(z, z_ld, HP, es, true) ||
+            !row_ok(B, B_ld, GN, es, true) || !row_ok(C, C_ld, GN, es, true) ||
+            !row_ok(y, y_ld, HP, es, true) || !row_ok(dt, dt_ld, d->nheads, es, false))
+            return SSD_ERR_UNSUPPORTED;
+    }
+    ssd::PrefillParams p{};
+    p.b = d->batch; p.L = d->seqlen;
+    p.H = d->nheads; p.P = d->headdim; p.G = d->ngroups; p.N = d->dstate; p.K = d->dconv;
+    p.Q = d->chunk; p.eps = d->eps; p.act = d->act;
+    p.nc = (p.L + p.Q - 1) / p.Q;
+    p.x = x; p.z = z; p.B = B; p.C = C; p.dt = dt;
+    p.x_ld = x_ld; p.z_ld = z_ld; p.B_ld = B_ld; p.C_ld = C_ld; p.dt_ld = dt_ld;
+    p.A = A; p.D = D; p.conv_w = conv_w; p.conv_b = conv_b; p.dt_bias = dt_bias; p.norm_w = norm_w;
+    p.init_ssm = init_ssm_state; p.init_conv = init_conv_state;
+    p.y = y; p.y_ld = y_ld; p.final_ssm = final_ssm_state; p.final_conv = final_conv_state;
+    char* ws = (char*)workspace;
+    p.status = (int*)(ws + wl.status);
+    p.xbc = ws + wl.xbc;
+    p.delta = (float*)(ws + wl.delta);
+    p.lam = (float*)(ws + wl.lam);
+    p.states = (float*)(ws + wl.states);
+    p.ypre = (float*)(ws + wl.ypre);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(p.status, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (ssd::launch_prefill_simt(p, st) != cudaSuccess) return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+ssd_status ssd_mixer_decode_step(const ssd_dims* d, const void* x, int64_t x_ld, const void* z,
+                                 int64_t z_ld, const void* B, int64_t B_ld, const void* C,
+                                 int64_t C_ld, const void* dt, int64_t dt_ld, const float* A,
+                                 const float* D, const float* conv_w, const float* conv_b,
+                                 const float* dt_bias, const float* norm_w, float* ssm_state,
+                                 void* conv_state, const int32_t* slot_idx, void* y, int64_t y_ld,
+                                 void* stream)
+{
+    const ssd_status ds = check_dims(d, true);
+    if (ds != SSD_OK) return ds;
+    if (d->batch == 0) return SSD_OK;
+    const size_t es = d->act == SSD_BF16 ? 2 : 4;
+    const int64_t HP = (int64_t)d->nheads * d->headdim, GN = (int64_t)d->ngroups * d->dstate;
+    if (!A || !D || !conv_w || !conv_b || !dt_bias || !norm_w || !ssm_state || !conv_state ||
+        !x || !z || !B || !C || !dt || !y)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(conv_w) || !aligned16(ssm_state) || ((uintptr_t)conv_state % es) ||
+        (slot_idx && ((uintptr_t)slot_idx & 3u)))
+        return SSD_ERR_UNSUPPORTED;
+    if (!row_ok(x, x_ld, HP, es, false) || !row_ok(z, z_ld, HP, es, false) ||
+        !row_ok(B, B_ld, GN, es, false) || !row_ok(C, C_ld, GN, es, false) ||
+        !row_ok(y, y_ld, HP, es, false) || !row_ok(dt, dt_ld, d->nheads, es, false))
+        return SSD_ERR_UNSUPPORTED;
+    ssd::DecodeParams p{};
+    p.b = d->batch;
+    p.H = d->nheads; p.P = d->headdim; p.G = d->ngroups; p.N = d->dstate; p.K = d->dconv;
+    p.eps = d->eps; p.act = d->act;
+    p.x = x; p.z = z; p.B = B; p.C = C; p.dt = dt;
+    p.x_ld = x_ld; p.z_ld = z_ld; p.B_ld = B_ld; p.C_ld = C_ld; p.dt_ld = dt_ld;
+    p.A = A; p.D = D; p.conv_w = conv_w; p.conv_b = conv_b; p.dt_bias = dt_bias; p.norm_w = norm_w;
+    p.ssm_state = ssm_state; p.conv_state = conv_state; p.slot_idx = slot_idx;
+    p.y = y; p.y_ld = y_ld;
+    if (ssd::launch_decode_step(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream)
+{
+    if (!workspace || ((uintptr_t)workspace & 255u)) return SSD_ERR_INVALID_ARG;
+    int v = 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+    return v == 0 ? SSD_OK : SSD_ERR_TIMEOUT;
+}
+
+const char* ssd_status_string(ssd_status s)
+{
+    switch (s) {
+    case SSD_OK: return "ok";
+    case SSD_ERR_INVALID_ARG: return "invalid argument";
+    case SSD_ERR_UNSUPPORTED: return "unsupported shape, alignment or dtype";
+    case SSD_ERR_CUDA: return "CUDA launch or runtime error";
+    case SSD_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+int ssd_mixer_version(void) { return 100; }
+
+}  // extern "C"

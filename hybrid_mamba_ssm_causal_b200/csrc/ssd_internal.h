@@ -1,0 +1,77 @@
+// ssd_internal.h -- launch parameters shared by the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __CUDACC__
+#define SSD_HD __host__ __device__
+#else
+#define SSD_HD
+#endif
+
+namespace ssd {
+
+// Everything one prefill call needs, validated by the ABI layer.
+struct PrefillParams {
+    int64_t b, L;        // batch rows, tokens per row
+    int H, P, G, N, K, Q;
+    float eps;
+    int act;             // 0 = fp32, 1 = bf16
+    int64_t nc;          // chunks per row = ceil(L / Q)
+    const void *x, *z, *B, *C, *dt;
+    int64_t x_ld, z_ld, B_ld, C_ld, dt_ld;
+    const float *A, *D, *conv_w, *conv_b, *dt_bias, *norm_w;
+    const float* init_ssm;   // [b][H][P][N] or nullptr
+    const void* init_conv;   // [b][Cc][K-1] or nullptr
+    void* y;
+    int64_t y_ld;
+    float* final_ssm;
+    void* final_conv;
+    // workspace regions (carved by the ABI layer)
+    int* status;     // device status word
+    void* xbc;       // [b][L][Cc] activated x|B|C, activation dtype
+    float* delta;    // [b][H][L]
+    float* lam;      // [b][H][L] within-chunk inclusive cumsum of delta*A
+    float* states;   // [b][nc][H][P][N] chunk states, then states entering each chunk
+    float* ypre;     // [b][L][HP] y before the gate and norm
+
+    SSD_HD int64_t HP() const { return (int64_t)H * P; }
+    SSD_HD int64_t GN() const { return (int64_t)G * N; }
+    SSD_HD int64_t Cc() const { return HP() + 2 * GN(); }
+};
+
+struct DecodeParams {
+    int64_t b;
+    int H, P, G, N, K;
+    float eps;
+    int act;
+    const void *x, *z, *B, *C, *dt;
+    int64_t x_ld, z_ld, B_ld, C_ld, dt_ld;
+    const float *A, *D, *conv_w, *conv_b, *dt_bias, *norm_w;
+    float* ssm_state;
+    void* conv_state;
+    const int32_t* slot_idx;
+    void* y;
+    int64_t y_ld;
+
+    SSD_HD int64_t HP() const { return (int64_t)H * P; }
+    SSD_HD int64_t GN() const { return (int64_t)G * N; }
+    SSD_HD int64_t Cc() const { return HP() + 2 * GN(); }
+};
+
+// Workspace layout of one prefill call; offsets in bytes, each 256-byte aligned.
+struct WorkspaceLayout {
+    size_t status, xbc, delta, lam, states, ypre, total;
+};
+WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
+                                         int act);
+
+bool prefill_simt_supported(int P, int N);
+cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t stream);
+
+bool decode_supported(int P, int N);
+cudaError_t launch_decode_step(const DecodeParams& p, cudaStream_t stream);
+
+}  // namespace ssd

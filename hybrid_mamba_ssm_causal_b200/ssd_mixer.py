@@ -1,0 +1,229 @@
+"""Thin Python binding of the C ABI in include/ssd_mixer.h (argument marshalling only).
+
+Every step of the mixer runs in libssd_mixer.so; this module only turns torch tensors
+into device pointers, leading dimensions and the current CUDA stream. There is no
+fallback: if the library is missing or the tensors are not on a CUDA device, the call
+raises.
+
+The entry points keep the C names:
+  ssd_mixer_prefill_workspace_size(dims) -> int
+  ssd_mixer_prefill(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                    init_ssm_state, init_conv_state, y, final_ssm_state, final_conv_state,
+                    workspace, stream=None)
+  ssd_mixer_decode_step(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                        ssm_state, conv_state, slot_idx, y, stream=None)
+plus :func:`prefill` / :func:`decode_step`, which allocate the outputs and workspace
+with torch and call the entry points above.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssd_mixer.so")
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
+SSD_F32, SSD_BF16 = 0, 1
+SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_decode_step",
+           "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version")
+
+
+class SsdError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{msg} (status {status})")
+        self.status = status
+
+
+class _CDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int32), ("headdim", ctypes.c_int32),
+                ("ngroups", ctypes.c_int32), ("dstate", ctypes.c_int32),
+                ("dconv", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("eps", ctypes.c_float), ("act", ctypes.c_int32)]
+
+
+@dataclass(frozen=True)
+class Dims:
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    ngroups: int
+    dstate: int
+    chunk: int = 128
+    dconv: int = 4
+    eps: float = 1e-5
+    act: str = "bf16"
+
+    @property
+    def d_inner(self) -> int:
+        return self.nheads * self.headdim
+
+    @property
+    def xbc_channels(self) -> int:
+        return self.d_inner + 2 * self.ngroups * self.dstate
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.act == "bf16" else torch.float32
+
+    def c(self) -> _CDims:
+        return _CDims(self.batch, self.seqlen, self.nheads, self.headdim, self.ngroups,
+                      self.dstate, self.dconv, self.chunk, self.eps,
+                      SSD_BF16 if self.act == "bf16" else SSD_F32)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Open libssd_mixer.so (raises if it is absent: build it with
+    ``python -m hybrid_mamba_ssm_causal_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} is missing "
+                           "(run python -m hybrid_mamba_ssm_causal_b200.build)")
+    lib = ctypes.CDLL(path)
+    V, I64, P = ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p
+    FP = ctypes.c_void_p
+    lib.ssd_mixer_prefill_workspace_size.argtypes = [ctypes.POINTER(_CDims)]
+    lib.ssd_mixer_prefill_workspace_size.restype = ctypes.c_size_t
+    lib.ssd_mixer_prefill.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
+                                      [FP, P, P, I64, FP, P, P, ctypes.c_size_t, V])
+    lib.ssd_mixer_prefill.restype = ctypes.c_int
+    lib.ssd_mixer_decode_step.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
+                                          [FP, P, P, P, I64, V])
+    lib.ssd_mixer_decode_step.restype = ctypes.c_int
+    lib.ssd_mixer_workspace_status.argtypes = [P, V]
+    lib.ssd_mixer_workspace_status.restype = ctypes.c_int
+    lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_mixer_version.argtypes = []
+    lib.ssd_mixer_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != SSD_OK:
+        raise SsdError(status, f"{what}: {load_library().ssd_status_string(status).decode()}")
+
+
+def _dev(t, name):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    return t.data_ptr()
+
+
+def _rows(t: torch.Tensor, name: str, rows: int, width: int):
+    """Pointer and leading dimension of a [.., rows, width]-shaped activation view whose
+    consecutive rows (tokens) are ``ld`` elements apart and whose last dim is unit-stride."""
+    if t.dim() < 2 or t.shape[-1] != width or t.stride(-1) != 1:
+        raise ValueError(f"{name}: expected last dim {width} with unit stride, got {tuple(t.shape)}")
+    if t.numel() // width != rows:
+        raise ValueError(f"{name}: expected {rows} rows, got {t.numel() // width}")
+    ld = t.stride(-2)
+    # all leading dims must be an even tiling by ld (token t of row i at (i*L + t) * ld)
+    expect = ld
+    for d in range(t.dim() - 2, -1, -1):
+        if t.shape[d] > 1 and t.stride(d) != expect:
+            raise ValueError(f"{name}: rows must be evenly strided")
+        expect *= t.shape[d]
+    return _dev(t, name), ld
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def ssd_mixer_prefill_workspace_size(dims: Dims) -> int:
+    cd = dims.c()
+    return int(load_library().ssd_mixer_prefill_workspace_size(ctypes.byref(cd)))
+
+
+def ssd_mixer_prefill(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                      init_ssm_state, init_conv_state, y, final_ssm_state, final_conv_state,
+                      workspace, stream=None) -> None:
+    lib = load_library()
+    rows = dims.batch * dims.seqlen
+    HP, GN = dims.d_inner, dims.ngroups * dims.dstate
+    args = []
+    for t, name, w in ((x, "x", HP), (z, "z", HP), (B, "B", GN), (C, "C", GN), (dt, "dt", dims.nheads)):
+        args += list(_rows(t, name, rows, w))
+    py, y_ld = _rows(y, "y", rows, HP)
+    cd = dims.c()
+    st = lib.ssd_mixer_prefill(
+        ctypes.byref(cd), *args, _dev(A, "A"), _dev(D, "D"), _dev(conv_w, "conv_w"),
+        _dev(conv_b, "conv_b"), _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"),
+        _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
+        py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "ssd_mixer_prefill")
+
+
+def ssd_mixer_decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                          ssm_state, conv_state, slot_idx, y, stream=None) -> None:
+    lib = load_library()
+    HP, GN = dims.d_inner, dims.ngroups * dims.dstate
+    args = []
+    for t, name, w in ((x, "x", HP), (z, "z", HP), (B, "B", GN), (C, "C", GN), (dt, "dt", dims.nheads)):
+        args += list(_rows(t, name, dims.batch, w))
+    py, y_ld = _rows(y, "y", dims.batch, HP)
+    if slot_idx is not None and slot_idx.dtype != torch.int32:
+        raise TypeError("slot_idx must be int32")
+    cd = dims.c()
+    st = lib.ssd_mixer_decode_step(
+        ctypes.byref(cd), *args, _dev(A, "A"), _dev(D, "D"), _dev(conv_w, "conv_w"),
+        _dev(conv_b, "conv_b"), _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"),
+        _dev(ssm_state, "ssm_state"), _dev(conv_state, "conv_state"), _dev(slot_idx, "slot_idx"),
+        py, y_ld, _stream(stream))
+    _check(st, "ssd_mixer_decode_step")
+
+
+def ssd_mixer_workspace_status(workspace, stream=None) -> int:
+    return int(load_library().ssd_mixer_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
+
+
+def alloc_workspace(dims: Dims, device="cuda") -> torch.Tensor:
+    n = ssd_mixer_prefill_workspace_size(dims)
+    if n == 0:
+        raise SsdError(SSD_ERR_UNSUPPORTED, "ssd_mixer_prefill_workspace_size: unsupported dims")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def prefill(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+            init_ssm_state=None, init_conv_state=None, workspace=None, out=None, stream=None):
+    """Allocate y, the final states and (if not given) the workspace, then run
+    :func:`ssd_mixer_prefill`. Returns (y, final_ssm_state, final_conv_state)."""
+    dev = x.device
+    b, L, H, P, N = dims.batch, dims.seqlen, dims.nheads, dims.headdim, dims.dstate
+    if out is None:
+        y = torch.empty(b, L, dims.d_inner, dtype=dims.torch_dtype, device=dev)
+        fs = torch.empty(b, H, P, N, dtype=torch.float32, device=dev)
+        fc = torch.empty(b, dims.xbc_channels, dims.dconv - 1, dtype=dims.torch_dtype, device=dev)
+    else:
+        y, fs, fc = out
+    ws = workspace if workspace is not None else alloc_workspace(dims, dev)
+    ssd_mixer_prefill(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                      init_ssm_state, init_conv_state, y, fs, fc, ws, stream)
+    return y, fs, fc
+
+
+def decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                ssm_state, conv_state, slot_idx=None, y=None, stream=None):
+    """Run :func:`ssd_mixer_decode_step` (states updated in place); returns y."""
+    if y is None:
+        y = torch.empty(dims.batch, dims.d_inner, dtype=dims.torch_dtype, device=x.device)
+    ssd_mixer_decode_step(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                          ssm_state, conv_state, slot_idx, y, stream)
+    return y

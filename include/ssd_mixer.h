@@ -1,0 +1,168 @@
+/*
+ * ssd_mixer.h -- C ABI of a B200 (sm_100a) library for the core of the Mamba-2
+ * mixer in Nemotron-H hybrid models: everything between in_proj and out_proj.
+ *
+ * The mixer projects its input (in_proj), runs a causal depthwise conv, the
+ * selective SSM scan and a gated RMSNorm, and projects back (out_proj); the
+ * recurrent state of each sequence lives in an engine slot (gllm PR #86 "feat(model): Nemotron-H hybrid (Mamba2 + attention + MoE) on the
+ * CPU", section "2. feat(model): Nemotron-H on the CPU", mixer table row M). The
+ * scan is the chunked "structured state-space duality" (SSD) form of the Mamba-2
+ * recurrence (openNemo model card, section "Architecture"; Modalities PR #459,
+ * section "Testing" and the ssd.py notes on the chunk-parallel block
+ * decomposition and the GatedRMSNorm semantics).
+ *
+ * Notation: b batch rows, L tokens per row, H heads, P head dim, G groups sharing
+ * B and C, N state dim, K conv width (4), HP = H*P, GN = G*N, Cc = HP + 2*GN (the
+ * xBC channels), r = H/G heads per group; head h reads group h / r.
+ *
+ * What every call computes, per batch row, for t = 0..L-1:
+ *   xBC' = SiLU(causal depthwise conv_K([x|B|C]) + conv_b), the conv running over
+ *          the K-1 stored raw inputs followed by this call's inputs;
+ *   delta_t[h] = softplus(dt_t[h] + dt_bias[h]);
+ *   h_t = exp(delta_t[h] * A[h]) * h_{t-1} + delta_t[h] * x'_t[h] (outer) B'_t[g];
+ *   y_t[h] = h_t . C'_t[g] + D[h] * x'_t[h];
+ *   out_t  = RMSNorm over each contiguous group of HP/G channels of
+ *            (y_t * SiLU(z_t)), times norm_w, with eps.
+ * The prefill evaluates the scan chunk by chunk (chunk = Q tokens): exact up to
+ * rounding, whatever Q is.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE pointers owned by the caller, except `dims`, which is a
+ *    host pointer read during the call only. The library allocates nothing, keeps
+ *    no pointer after the call returns and never synchronises the stream.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and runs asynchronously. Results are ready when the stream is.
+ *  - Activations (x, z, B, C, dt, y and the conv state) have dtype dims->act: fp32
+ *    or bf16. Parameters (A, D, conv_w, conv_b, dt_bias, norm_w) and the SSM state
+ *    are always fp32. Arithmetic is fp32 throughout; bf16 activations feed the
+ *    tensor-core contractions as bf16 with fp32 accumulation.
+ *  - Row layouts: token t of batch row i of x starts at x + (i*L + t) * x_ld
+ *    elements (likewise z, B, C, dt, y with their own ld), so the five inputs may
+ *    be column slices of one packed in_proj output. x, z, B, C and y must be
+ *    16-byte aligned with ld*elem_size a multiple of 16 bytes; dt needs only
+ *    element alignment. x and y must not overlap.
+ *  - Parameter layouts: A, D, dt_bias [H] (A negative); conv_w [Cc][K] with tap K-1
+ *    on the current token; conv_b [Cc]; norm_w [HP]; channel order of Cc is x
+ *    (HP), then B (GN), then C (GN).
+ *  - State layouts: SSM state [slots or b][H][P][N] fp32, N contiguous; conv state
+ *    [slots or b][Cc][K-1] in the activation dtype, oldest raw input first.
+ *  - Errors: argument errors return SSD_ERR_INVALID_ARG or SSD_ERR_UNSUPPORTED
+ *    before anything is launched; a failed launch returns SSD_ERR_CUDA. Nothing
+ *    is written when an error is returned before the launch.
+ */
+#ifndef SSD_MIXER_H
+#define SSD_MIXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,  /* null pointer, bad size, workspace too small */
+    SSD_ERR_UNSUPPORTED = 2,  /* shape/alignment/dtype this build does not run */
+    SSD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
+    SSD_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (status word) */
+} ssd_status;
+
+typedef enum ssd_dtype {
+    SSD_F32 = 0,
+    SSD_BF16 = 1,
+} ssd_dtype;
+
+/* Problem dimensions (a plain struct; every field is read, none is kept). */
+typedef struct ssd_dims {
+    int64_t batch;    /* b: batch rows (prefill) or sequences stepped (decode) */
+    int64_t seqlen;   /* L: tokens per row in this call (decode: must be 1)     */
+    int32_t nheads;   /* H */
+    int32_t headdim;  /* P: 16, 32, 64 or 128 */
+    int32_t ngroups;  /* G: divides H */
+    int32_t dstate;   /* N: 16, 32, 64 or 128 */
+    int32_t dconv;    /* K: must be 4 */
+    int32_t chunk;    /* Q: prefill chunk length, 16..256 and a multiple of 16 */
+    float eps;        /* RMSNorm epsilon (> 0) */
+    int32_t act;      /* ssd_dtype of the activations */
+} ssd_dims;
+
+/* Bytes of device workspace ssd_mixer_prefill needs for `dims`; 0 when the dims
+ * are invalid or unsupported (call ssd_mixer_prefill to learn which). The size
+ * grows linearly with batch * seqlen. */
+SSD_API size_t ssd_mixer_prefill_workspace_size(const ssd_dims* dims);
+
+/* Prefill: run L tokens of b independent rows through the mixer core.
+ *
+ * Inputs: x, z [b][L][HP]; B, C [b][L][GN]; dt [b][L][H] (raw, before the bias);
+ * parameters as above; init_ssm_state [b][H][P][N] and init_conv_state [b][Cc][K-1]
+ * (either may be NULL = zeros). To continue a sequence that arrives in several
+ * pieces, pass the previous call's final states as this call's initial states (the
+ * split-prefill case of gllm PR #86, section "Validation").
+ * Outputs: y [b][L][HP] (gated, normalised; y_ld), final_ssm_state, final_conv_state
+ * (same layouts as the inits). A final state may be the same buffer as its init.
+ * workspace: device scratch of at least ssd_mixer_prefill_workspace_size(dims)
+ * bytes, 256-byte aligned, not shared with a concurrently running call.
+ * L = 0 is allowed: y is untouched and the final states equal the initial ones. */
+SSD_API ssd_status ssd_mixer_prefill(const ssd_dims* dims,
+                             const void* x, int64_t x_ld,
+                             const void* z, int64_t z_ld,
+                             const void* B, int64_t B_ld,
+                             const void* C, int64_t C_ld,
+                             const void* dt, int64_t dt_ld,
+                             const float* A, const float* D,
+                             const float* conv_w, const float* conv_b,
+                             const float* dt_bias, const float* norm_w,
+                             const float* init_ssm_state, const void* init_conv_state,
+                             void* y, int64_t y_ld,
+                             float* final_ssm_state, void* final_conv_state,
+                             void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Decode step: advance b sequences by one token each, in place on their state
+ * slots (the one-token-at-a-time decode of gllm PR #86, section "Validation", where
+ * each Mamba layer picks up from the state held in the sequence's slot).
+ *
+ * dims->seqlen must be 1 and dims->chunk is ignored. x, z [b][HP]; B, C [b][GN];
+ * dt [b][H] with row strides x_ld ... dt_ld between sequences.
+ * ssm_state [nslots][H][P][N] fp32 and conv_state [nslots][Cc][K-1] are read and
+ * rewritten in place for the slots named by slot_idx [b] (int32, device; NULL =
+ * sequence i uses slot i). Slot indices must be distinct and in range; the library
+ * cannot check device-resident indices. y [b][HP] (y_ld) receives the output. */
+SSD_API ssd_status ssd_mixer_decode_step(const ssd_dims* dims,
+                                 const void* x, int64_t x_ld,
+                                 const void* z, int64_t z_ld,
+                                 const void* B, int64_t B_ld,
+                                 const void* C, int64_t C_ld,
+                                 const void* dt, int64_t dt_ld,
+                                 const float* A, const float* D,
+                                 const float* conv_w, const float* conv_b,
+                                 const float* dt_bias, const float* norm_w,
+                                 float* ssm_state, void* conv_state,
+                                 const int32_t* slot_idx,
+                                 void* y, int64_t y_ld,
+                                 void* stream);
+
+/* Reads the device status word that the prefill kernels keep at the start of
+ * `workspace` (written by the last call that used it). Synchronises `stream`.
+ * Returns SSD_OK, or SSD_ERR_TIMEOUT if a bounded device-side wait gave up, in
+ * which case that call's outputs are invalid. */
+SSD_API ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream);
+
+/* Static description of a status code (never NULL). */
+SSD_API const char* ssd_status_string(ssd_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+SSD_API int ssd_mixer_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_MIXER_H */

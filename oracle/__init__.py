@@ -198,9 +198,8 @@ def decode_step(d: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
                 ssm_state, conv_state, slot_idx=None, nthreads: int | None = None):
     """One single-token decode step on state slots (returns y [b, H*P] and NEW state
     arrays; inputs are not modified). A decode step is the prefill of one token that
-    resumes from the slot's states and leaves its final states in the slot (gllm PR
-    #86, section "Validation": token-by-token decode, every Mamba layer resuming from
-    its slot)."""
+    starts from the slot's states and leaves its final states in the slot (the
+    one-token-at-a-time decode case of gllm PR #86, section "Validation")."""
     b = np.asarray(x).shape[0]
     slots = np.arange(b) if slot_idx is None else np.asarray(slot_idx)
     d1 = Dims(b, 1, d.nheads, d.headdim, d.ngroups, d.dstate, d.dconv, d.eps)

@@ -6,15 +6,15 @@
  * __graft_entry__.py and the cpu_baseline / reference leg of bench.py may load
  * it. It shares no code, header, table or helper with the CUDA path.
  *
- * What it computes (everything between in_proj and out_proj of a Nemotron-H
- * Mamba-2 layer: "in_proj, then CausalConv1D, SSMScan and GatedRMSNorm, then
- * out_proj" -- gllm PR #86 "feat(model): Nemotron-H hybrid (Mamba2 + attention
- * + MoE) on the CPU", section "2. feat(model): Nemotron-H on the CPU", mixer
- * table, row M):
+ * What it computes: everything between in_proj and out_proj of a Nemotron-H
+ * Mamba-2 layer, i.e. the causal conv, the selective SSM scan and the gated norm
+ * that the mixer table of gllm PR #86 "feat(model): Nemotron-H hybrid (Mamba2 +
+ * attention + MoE) on the CPU" (section "2. feat(model): Nemotron-H on the CPU",
+ * row M) places between the two projections:
  *
- *   1. xBC = [x | B | C] on the channel axis (the fused projection emits
- *      "[z | xBC | dt]" -- same PR, "Supporting changes"; Modalities PR #459,
- *      packed "[z, x, B, C, dt]" projection layout).
+ *   1. xBC = [x | B | C] on the channel axis (the fused projection's output row
+ *      holds z, then x, B and C, then dt -- same PR, "Supporting changes";
+ *      Modalities PR #459, notes on the packed projection layout).
  *   2. Depthwise causal conv of width K over time, per channel c:
  *        s    = [init_conv[c][0..K-2] (oldest first), xBC[0..L-1][c]]
  *        v[t] = conv_b[c] + sum_{k=0}^{K-1} conv_w[c][k] * s[t+k]

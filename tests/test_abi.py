@@ -1,0 +1,106 @@
+"""The C ABI loads, exports every declared symbol, and refuses bad arguments before any
+launch (CPU only: every case here fails validation, so nothing reaches a GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from hybrid_mamba_ssm_causal_b200 import build as build_mod
+from hybrid_mamba_ssm_causal_b200 import ssd_mixer as sm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return sm.load_library()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names |= set(re.findall(r"SSD_API\s+[\w\s\*]+?\b(\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("ssd_mixer_prefill", "ssd_mixer_decode_step", "ssd_mixer_prefill_workspace_size",
+              "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_symbols():
+        assert hasattr(lib, n), f"missing export {n}"
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.ssd_status_string(s)
+    assert lib.ssd_mixer_version() >= 100
+
+
+def _dims(**kw):
+    base = dict(batch=2, seqlen=64, nheads=4, headdim=16, ngroups=2, dstate=16, chunk=64, act="bf16")
+    base.update(kw)
+    return sm.Dims(**base)
+
+
+FAKE = 1 << 40  # a 256-byte-aligned address that is never dereferenced
+
+
+def call_prefill(lib, d, ptr=FAKE, ws_bytes=1 << 30, x_ld=None, chunk_ws=None):
+    cd = d.c()
+    HP, GN = d.d_inner, d.ngroups * d.dstate
+    P = ctypes.c_void_p
+    return lib.ssd_mixer_prefill(ctypes.byref(cd), ptr, x_ld or HP, FAKE, HP, FAKE, GN, FAKE, GN,
+                                 FAKE, d.nheads, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                 FAKE, HP, FAKE, FAKE, FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(dconv=3), sm.SSD_ERR_UNSUPPORTED),
+    (dict(chunk=100), sm.SSD_ERR_UNSUPPORTED),
+    (dict(chunk=8), sm.SSD_ERR_UNSUPPORTED),
+    (dict(headdim=24), sm.SSD_ERR_UNSUPPORTED),
+    (dict(dstate=256), sm.SSD_ERR_UNSUPPORTED),
+    (dict(ngroups=3), sm.SSD_ERR_INVALID_ARG),
+    (dict(eps=0.0), sm.SSD_ERR_INVALID_ARG),
+    (dict(batch=-1), sm.SSD_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_bad_dims(lib, bad, status):
+    assert call_prefill(lib, _dims(**bad)) == status
+    assert lib.ssd_mixer_prefill_workspace_size(ctypes.byref(_dims(**bad).c())) == 0
+
+
+def test_prefill_rejects_misaligned_rows(lib):
+    assert call_prefill(lib, _dims(), ptr=FAKE + 2) == sm.SSD_ERR_UNSUPPORTED
+    assert call_prefill(lib, _dims(), x_ld=64 + 1) == sm.SSD_ERR_UNSUPPORTED
+
+
+def test_prefill_rejects_small_workspace(lib):
+    d = _dims()
+    need = lib.ssd_mixer_prefill_workspace_size(ctypes.byref(d.c()))
+    assert need > 0
+    assert call_prefill(lib, d, ws_bytes=need - 1) == sm.SSD_ERR_INVALID_ARG
+
+
+def test_decode_rejects_seqlen_not_one(lib):
+    d = _dims(seqlen=2)
+    cd = d.c()
+    HP, GN = d.d_inner, d.ngroups * d.dstate
+    st = lib.ssd_mixer_decode_step(ctypes.byref(cd), FAKE, HP, FAKE, HP, FAKE, GN, FAKE, GN, FAKE,
+                                   d.nheads, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                   FAKE, HP, None)
+    assert st == sm.SSD_ERR_INVALID_ARG
+
+
+def test_workspace_size_grows_with_tokens(lib):
+    a = lib.ssd_mixer_prefill_workspace_size(ctypes.byref(_dims(seqlen=64).c()))
+    b = lib.ssd_mixer_prefill_workspace_size(ctypes.byref(_dims(seqlen=640).c()))
+    assert b > 5 * a
