@@ -131,7 +131,6 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.states = (float*)(ws + wl.states);
     p.ypre = (float*)(ws + wl.ypre);
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(p.status, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::launch_prefill_simt(p, st) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }

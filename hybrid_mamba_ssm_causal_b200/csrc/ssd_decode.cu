@@ -19,6 +19,7 @@
 //   4. gated RMSNorm over the group's r*P channels; y written in the activation dtype.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_profile.h"
 
 namespace ssd {
 namespace {
@@ -152,6 +153,7 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t st)
         cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<T, NN>,                           \
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
         if (e != cudaSuccess) return e;                                                           \
+        LaunchScope ls("decode_step", st);                                                        \
         decode_step_kernel<T, NN><<<grid, kThreads, smem, st>>>(p);                               \
         return cudaGetLastError();                                                                \
     }

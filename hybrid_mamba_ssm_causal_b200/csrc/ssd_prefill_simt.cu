@@ -22,6 +22,7 @@
 // tensor-core path.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_profile.h"
 
 namespace ssd {
 namespace {
@@ -95,6 +96,7 @@ __global__ void conv_state_kernel(PrefillParams p)
 {
     const int64_t HP = p.HP(), GN = p.GN(), Cc = p.Cc();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx == 0) *p.status = 0;  // this call's status word starts clean
     if (idx >= p.b * Cc) return;
     const int64_t bi = idx / Cc, c = idx % Cc;
     const T* src;
@@ -388,14 +390,21 @@ __global__ void __launch_bounds__(256) gated_norm_kernel(PrefillParams p)
 template <typename T, int P, int N>
 cudaError_t launch_scan_kernels(const PrefillParams& p, cudaStream_t st)
 {
-    chunk_state_kernel<T, P, N><<<dim3((unsigned)p.nc, p.H, (unsigned)p.b), 256, 0, st>>>(p);
+    {
+        LaunchScope ls("simt_chunk_state", st);
+        chunk_state_kernel<T, P, N><<<dim3((unsigned)p.nc, p.H, (unsigned)p.b), 256, 0, st>>>(p);
+    }
     const int64_t PN = (int64_t)P * N;
-    state_pass_kernel<<<dim3((unsigned)((PN / 4 + 255) / 256), p.H, (unsigned)p.b), 256, 0, st>>>(p);
+    {
+        LaunchScope ls("simt_state_pass", st);
+        state_pass_kernel<<<dim3((unsigned)((PN / 4 + 255) / 256), p.H, (unsigned)p.b), 256, 0, st>>>(p);
+    }
     const size_t smem = sizeof(ScanSmem<P, N>);
     cudaError_t e = cudaFuncSetAttribute(chunk_scan_kernel<T, P, N>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (p.Q + kTile - 1) / kTile;
+    LaunchScope ls("simt_chunk_scan", st);
     chunk_scan_kernel<T, P, N><<<dim3((unsigned)(tiles * p.nc), p.H, (unsigned)p.b), 256, smem, st>>>(p);
     return cudaSuccess;
 }
@@ -406,12 +415,18 @@ cudaError_t launch_all(const PrefillParams& p, cudaStream_t st)
     constexpr int V = Act<T>::kVec;
     const int64_t Cc = p.Cc();
     if (p.b == 0) return cudaSuccess;
-    if (p.L > 0)
+    if (p.L > 0) {
+        LaunchScope ls("conv_silu", st);
         conv_silu_kernel<T><<<dim3((unsigned)((p.L + kConvTokens - 1) / kConvTokens),
                                    (unsigned)((Cc / V + 127) / 128), (unsigned)p.b), 128, 0, st>>>(p);
-    conv_state_kernel<T><<<(unsigned)((p.b * Cc + 255) / 256), 256, 0, st>>>(p);
+    }
+    {
+        LaunchScope ls("conv_state", st);
+        conv_state_kernel<T><<<(unsigned)((p.b * Cc + 255) / 256), 256, 0, st>>>(p);
+    }
     if (p.L == 0) {  // no tokens: the final SSM state is the initial one
         const int64_t PN = (int64_t)p.P * p.N;
+        LaunchScope ls("simt_state_pass", st);
         state_pass_kernel<<<dim3((unsigned)((PN / 4 + 255) / 256), p.H, (unsigned)p.b), 256, 0, st>>>(p);
         return cudaGetLastError();
     }
@@ -424,7 +439,10 @@ cudaError_t launch_all(const PrefillParams& p, cudaStream_t st)
 #undef SSD_SIMT_CASE
     if (e != cudaSuccess) return e;
     const int64_t warps = p.b * p.L * p.G;
-    gated_norm_kernel<T><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+    {
+        LaunchScope ls("gated_norm", st);
+        gated_norm_kernel<T><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+    }
     return cudaGetLastError();
 }
 

@@ -1,0 +1,87 @@
+// ssd_profile.cu -- launch counter and opt-in per-kernel event timing (see ssd_profile.h).
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/ssd_mixer.h"
+#include "ssd_profile.h"
+
+namespace ssd {
+namespace {
+
+struct Rec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+
+std::atomic<long long> g_launches{0};
+std::atomic<int> g_enabled{0};
+std::mutex g_mu;
+std::vector<Rec> g_recs;
+
+}  // namespace
+
+void profile_begin(const char* name, cudaStream_t st, void** token)
+{
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    *token = nullptr;
+    if (!g_enabled.load(std::memory_order_relaxed)) return;
+    Rec* r = new Rec{name, nullptr, nullptr};
+    if (cudaEventCreate(&r->a) != cudaSuccess || cudaEventCreate(&r->b) != cudaSuccess ||
+        cudaEventRecord(r->a, st) != cudaSuccess) {
+        delete r;
+        return;
+    }
+    *token = r;
+}
+
+void profile_end(void* token, cudaStream_t st)
+{
+    if (!token) return;
+    Rec* r = (Rec*)token;
+    cudaEventRecord(r->b, st);
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_recs.push_back(*r);
+    delete r;
+}
+
+}  // namespace ssd
+
+extern "C" {
+
+long long ssd_mixer_launch_count(void) { return ssd::g_launches.load(); }
+
+void ssd_mixer_profile_enable(int on) { ssd::g_enabled.store(on ? 1 : 0); }
+
+int ssd_mixer_profile_read(const char** names, double* total_ms, int* launches, int max_entries)
+{
+    std::vector<ssd::Rec> recs;
+    {
+        std::lock_guard<std::mutex> lk(ssd::g_mu);
+        recs.swap(ssd::g_recs);
+    }
+    int n = 0;
+    for (const ssd::Rec& r : recs) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            ms = -1.0f;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+        int k = 0;
+        while (k < n && strcmp(names[k], r.name) != 0) ++k;
+        if (k == n) {
+            if (n >= max_entries) continue;
+            names[n] = r.name;
+            total_ms[n] = 0.0;
+            launches[n] = 0;
+            ++n;
+        }
+        total_ms[k] += ms;
+        launches[k] += 1;
+    }
+    return n;
+}
+
+}  // extern "C"

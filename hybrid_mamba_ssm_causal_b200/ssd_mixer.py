@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(HERE, "libssd_mixer.so")
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
 SSD_F32, SSD_BF16 = 0, 1
 SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_decode_step",
-           "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version")
+           "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version",
+           "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read")
 
 
 class SsdError(RuntimeError):
@@ -106,6 +107,13 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_mixer_version.argtypes = []
     lib.ssd_mixer_version.restype = ctypes.c_int
+    lib.ssd_mixer_launch_count.argtypes = []
+    lib.ssd_mixer_launch_count.restype = ctypes.c_longlong
+    lib.ssd_mixer_profile_enable.argtypes = [ctypes.c_int]
+    lib.ssd_mixer_profile_enable.restype = None
+    lib.ssd_mixer_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                           ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+    lib.ssd_mixer_profile_read.restype = ctypes.c_int
     _lib = lib
     return lib
 

@@ -155,6 +155,24 @@ SSD_API ssd_status ssd_mixer_decode_step(const ssd_dims* dims,
  * which case that call's outputs are invalid. */
 SSD_API ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream);
 
+/* Number of kernels this library has launched in the process so far (all entry
+ * points, all devices). A caller reads it before and after a region to count the
+ * library's launches in that region. Not a compute call; thread-safe. */
+SSD_API long long ssd_mixer_launch_count(void);
+
+/* Switch per-kernel timing on (1) or off (0). While on, every kernel launch is
+ * bracketed by a pair of CUDA events recorded on the launching stream (a few
+ * microseconds of host overhead per launch; the kernels themselves are unchanged).
+ * Off by default. */
+SSD_API void ssd_mixer_profile_enable(int on);
+
+/* Collects the event pairs recorded since the last read: waits for each to complete
+ * and sums their elapsed times per kernel name. Writes up to max_entries rows into
+ * names (static strings owned by the library), total_ms and launches; returns the
+ * number of rows. Host arrays owned by the caller. */
+SSD_API int ssd_mixer_profile_read(const char** names, double* total_ms, int* launches,
+                                   int max_entries);
+
 /* Static description of a status code (never NULL). */
 SSD_API const char* ssd_status_string(ssd_status status);
 
