@@ -190,6 +190,7 @@ const char* ssd_status_string(ssd_status s)
     case SSD_ERR_UNSUPPORTED: return "unsupported shape, alignment or dtype";
     case SSD_ERR_CUDA: return "CUDA launch or runtime error";
     case SSD_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case SSD_ERR_TOO_LARGE: return "problem needs more scratch than the fixed static workspace holds";
     }
     return "unknown status";
 }

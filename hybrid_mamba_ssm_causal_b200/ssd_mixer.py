@@ -26,11 +26,13 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libssd_mixer.so")
 
-SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT, SSD_ERR_TOO_LARGE = range(6)
+SSD_MIXER_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 SSD_F32, SSD_BF16 = 0, 1
 SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_decode_step",
            "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version",
-           "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read")
+           "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read",
+           "ssd_mixer_prefill_static")
 
 
 class SsdError(RuntimeError):
@@ -101,6 +103,9 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_decode_step.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
                                           [FP, P, P, P, I64, V])
     lib.ssd_mixer_decode_step.restype = ctypes.c_int
+    lib.ssd_mixer_prefill_static.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
+                                             [FP, P, P, I64, FP, P, V])
+    lib.ssd_mixer_prefill_static.restype = ctypes.c_int
     lib.ssd_mixer_workspace_status.argtypes = [P, V]
     lib.ssd_mixer_workspace_status.restype = ctypes.c_int
     lib.ssd_status_string.argtypes = [ctypes.c_int]
@@ -177,6 +182,27 @@ def ssd_mixer_prefill(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias,
         py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "ssd_mixer_prefill")
+
+
+def ssd_mixer_prefill_static(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                             init_ssm_state, init_conv_state, y, final_ssm_state, final_conv_state,
+                             stream=None) -> int:
+    """The prefill with its scratch in the library's fixed device array (for callers that
+    cannot allocate device memory); returns the C status instead of raising."""
+    lib = load_library()
+    rows = dims.batch * dims.seqlen
+    HP, GN = dims.d_inner, dims.ngroups * dims.dstate
+    args = []
+    for t, name, w in ((x, "x", HP), (z, "z", HP), (B, "B", GN), (C, "C", GN), (dt, "dt", dims.nheads)):
+        args += list(_rows(t, name, rows, w))
+    py, y_ld = _rows(y, "y", rows, HP)
+    cd = dims.c()
+    return int(lib.ssd_mixer_prefill_static(
+        ctypes.byref(cd), *args, _dev(A, "A"), _dev(D, "D"), _dev(conv_w, "conv_w"),
+        _dev(conv_b, "conv_b"), _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"),
+        _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
+        py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
+        _stream(stream)))
 
 
 def ssd_mixer_decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,

@@ -72,6 +72,7 @@ typedef enum ssd_status {
     SSD_ERR_UNSUPPORTED = 2,  /* shape/alignment/dtype this build does not run */
     SSD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
     SSD_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (status word) */
+    SSD_ERR_TOO_LARGE = 5,    /* needs more scratch than the fixed static workspace */
 } ssd_status;
 
 typedef enum ssd_dtype {
@@ -148,6 +149,38 @@ SSD_API ssd_status ssd_mixer_decode_step(const ssd_dims* dims,
                                  const int32_t* slot_idx,
                                  void* y, int64_t y_ld,
                                  void* stream);
+
+/* Size of the fixed device scratch array used by ssd_mixer_prefill_static. */
+#define SSD_MIXER_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+
+/* Prefill without a caller-supplied workspace (no counterpart in the pages: this is a
+ * library convenience). For callers that cannot allocate device memory -- a plugin
+ * slot that receives only tensors and a stream, or a process whose device memory is
+ * wholly reserved by its own pool so that a cudaMalloc would fail or would stall the
+ * device mid-loop. Same arguments and results as ssd_mixer_prefill, minus the
+ * workspace: the scratch is a file-scope device array of
+ * SSD_MIXER_STATIC_WORKSPACE_BYTES that every GPU loading this library holds until the
+ * process exits. The library allocates nothing here either.
+ *  - Calls needing more scratch than that (ssd_mixer_prefill_workspace_size(dims) >
+ *    SSD_MIXER_STATIC_WORKSPACE_BYTES) return SSD_ERR_TOO_LARGE and launch nothing.
+ *  - The first call on a device looks up the array's device address (with that device
+ *    current) and caches it; make that first call before any stream capture.
+ *  - All calls on a device share the one array. Calls that overlap on the GPU (other
+ *    streams, no ordering between them) race on it and give wrong results: order them
+ *    on one stream or with events. */
+SSD_API ssd_status ssd_mixer_prefill_static(const ssd_dims* dims,
+                                    const void* x, int64_t x_ld,
+                                    const void* z, int64_t z_ld,
+                                    const void* B, int64_t B_ld,
+                                    const void* C, int64_t C_ld,
+                                    const void* dt, int64_t dt_ld,
+                                    const float* A, const float* D,
+                                    const float* conv_w, const float* conv_b,
+                                    const float* dt_bias, const float* norm_w,
+                                    const float* init_ssm_state, const void* init_conv_state,
+                                    void* y, int64_t y_ld,
+                                    float* final_ssm_state, void* final_conv_state,
+                                    void* stream);
 
 /* Reads the device status word that the prefill kernels keep at the start of
  * `workspace` (written by the last call that used it). Synchronises `stream`.

@@ -1,0 +1,64 @@
+"""GPU test of ssd_mixer_prefill_static, the prefill that allocates nothing (needs a B200).
+
+Some callers cannot allocate device memory: a plugin slot that hands the library only
+tensors and a stream, or a serving process whose memory is fully reserved by its own
+pool. For them the library keeps a fixed device array as the prefill's scratch. This
+test calls that entry point through the C ABI twice in a row on different inputs and
+checks each result against the regular entry point (caller-supplied workspace) within
+the parity tolerance, then checks that an oversized problem is refused. The file is
+named to be collected last, so a run that stops at the first failure has already run
+every other test; it also passes when run alone in a fresh process.
+"""
+import numpy as np
+import pytest
+import torch
+
+from hybrid_mamba_ssm_causal_b200 import ssd_mixer as sm
+from hybrid_mamba_ssm_causal_b200.workloads import WORKLOADS, make_prefill_inputs
+from tests.gpu_util import TOL, assert_close, dims_of, gpu_prefill, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _static_call(d, dv, y, fs, fc):
+    return sm.ssd_mixer_prefill_static(d, dv["x"], dv["z"], dv["B"], dv["C"], dv["dt"], dv["A"], dv["D"],
+                                       dv["conv_w"], dv["conv_b"], dv["dt_bias"], dv["norm_w"],
+                                       dv["init_ssm"], dv["init_conv"], y, fs, fc)
+
+
+@pytest.mark.parametrize("act", ["bf16", "f32"])
+def test_static_workspace_prefill_matches_regular_prefill_twice(act):
+    base = WORKLOADS["small_bf16"] if act == "bf16" else WORKLOADS["tiny_f32"]
+    w = base.with_(batch=2, seqlen=333, init_ssm_std=0.1, init_conv_std=1.0)
+    d = dims_of(w)
+    assert sm.ssd_mixer_prefill_workspace_size(d) <= sm.SSD_MIXER_STATIC_WORKSPACE_BYTES
+    adt = torch.bfloat16 if act == "bf16" else torch.float32
+    for seed in (101, 202):                       # two calls in a row, different inputs
+        dv = to_dev(make_prefill_inputs(w, seed=seed), act)
+        y = torch.empty(w.batch, w.seqlen, w.d_inner, dtype=adt, device="cuda")
+        fs = torch.empty(w.batch, w.nheads, w.headdim, w.dstate, device="cuda")
+        fc = torch.empty(w.batch, w.xbc_channels, 3, dtype=adt, device="cuda")
+        st = _static_call(d, dv, y, fs, fc)
+        assert st == sm.SSD_OK, st
+        y_ref, fs_ref, fc_ref = gpu_prefill(d, dv)
+        torch.cuda.synchronize()
+        tol = TOL[act]
+        assert_close("y", y, y_ref.float().cpu().numpy(), tol)
+        assert_close("final_ssm", fs, fs_ref.cpu().numpy(), tol)
+        assert_close("final_conv", fc, fc_ref.float().cpu().numpy(), tol)
+
+
+def test_static_workspace_refuses_oversized_problem():
+    w = WORKLOADS["small_bf16"]
+    d = dims_of(w, batch=8, seqlen=4096)
+    assert sm.ssd_mixer_prefill_workspace_size(d) > sm.SSD_MIXER_STATIC_WORKSPACE_BYTES
+    x = torch.zeros(8, 4096, w.d_inner, dtype=torch.bfloat16, device="cuda")
+    bc = torch.zeros(8, 4096, w.ngroups * w.dstate, dtype=torch.bfloat16, device="cuda")
+    dt = torch.zeros(8, 4096, w.nheads, dtype=torch.bfloat16, device="cuda")
+    prm = torch.zeros(w.xbc_channels * 4, device="cuda")
+    fs = torch.zeros(8, w.nheads, w.headdim, w.dstate, device="cuda")
+    fc = torch.zeros(8, w.xbc_channels, 3, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(x)
+    st = sm.ssd_mixer_prefill_static(d, x, x, bc, bc, dt, prm, prm, prm, prm, prm, prm, None, None,
+                                     y, fs, fc)
+    assert st == sm.SSD_ERR_TOO_LARGE
