@@ -143,6 +143,8 @@ def _rows(t: torch.Tensor, name: str, rows: int, width: int):
         raise ValueError(f"{name}: expected last dim {width} with unit stride, got {tuple(t.shape)}")
     if t.numel() // width != rows:
         raise ValueError(f"{name}: expected {rows} rows, got {t.numel() // width}")
+    if rows == 0:          # nothing is read or written; any row stride will do
+        return _dev(t, name), width
     ld = t.stride(-2)
     # all leading dims must be an even tiling by ld (token t of row i at (i*L + t) * ld)
     expect = ld
