@@ -14,6 +14,12 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
                                          int act)
 {
     WorkspaceLayout w{};
+    if (prefill_tc_supported(act, P, N, H, G)) {   // everything stays on chip
+        w.status = 0;
+        w.xbc = w.delta = w.lam = w.states = w.ypre = 256;
+        w.total = 256;
+        return w;
+    }
     const size_t es = act == SSD_BF16 ? 2 : 4;
     const int64_t HP = (int64_t)H * P, Cc = HP + 2 * (int64_t)G * N;
     const int64_t nc = Q > 0 ? (L + Q - 1) / Q : 0;
@@ -55,7 +61,9 @@ ssd_status check_dims(const ssd_dims* d, bool decode)
         if ((2 * r * d->headdim + 2 * d->dstate + r + 8) * 4 > 200 * 1024) return SSD_ERR_UNSUPPORTED;
     } else {
         if (d->chunk < 16 || d->chunk > 256 || d->chunk % 16 != 0) return SSD_ERR_UNSUPPORTED;
-        if (!ssd::prefill_simt_supported(d->headdim, d->dstate)) return SSD_ERR_UNSUPPORTED;
+        if (!ssd::prefill_simt_supported(d->headdim, d->dstate) &&
+            !ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups))
+            return SSD_ERR_UNSUPPORTED;
         const int64_t nc = (d->seqlen + d->chunk - 1) / d->chunk;
         if (nc * ((d->chunk + 63) / 64) > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
     }
@@ -131,7 +139,9 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.states = (float*)(ws + wl.states);
     p.ypre = (float*)(ws + wl.ypre);
     cudaStream_t st = (cudaStream_t)stream;
-    if (ssd::launch_prefill_simt(p, st) != cudaSuccess) return SSD_ERR_CUDA;
+    const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
+    if ((tc ? ssd::launch_prefill_tc(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
+        return SSD_ERR_CUDA;
     return SSD_OK;
 }
 

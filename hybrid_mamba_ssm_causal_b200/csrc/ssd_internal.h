@@ -68,6 +68,11 @@ struct WorkspaceLayout {
 WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
                                          int act);
 
+// Tensor-core path: bf16 activations, P = 64, N = 128, 2, 4 or 8 heads per group. It keeps
+// every intermediate on chip and needs only the status word of the workspace.
+bool prefill_tc_supported(int act, int P, int N, int H, int G);
+cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t stream);
+
 bool prefill_simt_supported(int P, int N);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t stream);
 
