@@ -16,8 +16,9 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
     WorkspaceLayout w{};
     if (prefill_tc_supported(act, P, N, H, G)) {   // everything stays on chip
         w.status = 0;
-        w.xbc = w.delta = w.lam = w.states = w.ypre = 256;
+        w.xbc = w.delta = w.lam = w.states = w.ypre = w.ssp = 256;
         w.total = 256;
+        if (prefill_tc_split(H, G)) w.total = align256(256 + (size_t)(b * L * H) * 2 * 4);
         return w;
     }
     const size_t es = act == SSD_BF16 ? 2 : 4;
@@ -30,6 +31,7 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
     w.lam = off;    off = align256(off + (size_t)(b * H * L) * 4);
     w.states = off; off = align256(off + (size_t)(b * nc * H) * (size_t)P * N * 4);
     w.ypre = off;   off = align256(off + (size_t)(b * L * HP) * 4);
+    w.ssp = off;
     w.total = off;
     return w;
 }
@@ -138,6 +140,7 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.lam = (float*)(ws + wl.lam);
     p.states = (float*)(ws + wl.states);
     p.ypre = (float*)(ws + wl.ypre);
+    p.ssp = (float*)(ws + wl.ssp);
     cudaStream_t st = (cudaStream_t)stream;
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
     if ((tc ? ssd::launch_prefill_tc(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)

@@ -36,6 +36,7 @@ struct PrefillParams {
     float* lam;      // [b][H][L] within-chunk inclusive cumsum of delta*A
     float* states;   // [b][nc][H][P][N] chunk states, then states entering each chunk
     float* ypre;     // [b][L][HP] y before the gate and norm
+    float* ssp;      // tensor-core path, groups wider than one cluster: [b][L][H][2] sums of g^2
 
     SSD_HD int64_t HP() const { return (int64_t)H * P; }
     SSD_HD int64_t GN() const { return (int64_t)G * N; }
@@ -63,7 +64,7 @@ struct DecodeParams {
 
 // Workspace layout of one prefill call; offsets in bytes, each 256-byte aligned.
 struct WorkspaceLayout {
-    size_t status, xbc, delta, lam, states, ypre, total;
+    size_t status, xbc, delta, lam, states, ypre, ssp, total;
 };
 WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
                                          int act);
@@ -71,6 +72,7 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
 // Tensor-core path: bf16 activations, P = 64, N = 128, 2, 4 or 8 heads per group. It keeps
 // every intermediate on chip and needs only the status word of the workspace.
 bool prefill_tc_supported(int act, int P, int N, int H, int G);
+bool prefill_tc_split(int H, int G);   // the group norm is finished by a second kernel
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t stream);
 
 bool prefill_simt_supported(int P, int N);

@@ -67,8 +67,8 @@ struct Layout {
     static constexpr uint32_t STAGE_BYTES = (uint32_t)kStageRows * SROW * 2;
     static constexpr uint32_t OFF_MISC = OFF_STAGE + ((STAGE_BYTES + 127) / 128) * 128;
     // misc floats
-    static constexpr uint32_t F_LAM = 0, F_DL = 128, F_SCAN = 256, F_SSH = 264, F_RED = 520,
-                              F_CW = F_RED + R * 128, F_CB = F_CW + SROW * 4, F_NW = F_CB + SROW,
+    static constexpr uint32_t F_LAM = 0, F_DL = 128, F_V = 256, F_SCAN = 384, F_RED = 392,
+                              F_CW = F_RED + R * 256, F_CB = F_CW + SROW * 4, F_NW = F_CB + SROW,
                               F_END = F_NW + kP;
     static constexpr uint32_t OFF_BAR = OFF_MISC + ((F_END * 4 + 15) / 16) * 16;
     static constexpr uint32_t TOTAL = OFF_BAR + 32;
@@ -89,7 +89,10 @@ __device__ __forceinline__ float scan128(float v, float* tot)
     return v + off;
 }
 
-template <int R>
+// R = CTAs per cluster (heads per cluster). SPLIT: the group has more heads than one
+// cluster holds (H/G > R); each CTA then writes the gated values and its per-token sums
+// of squares, and norm_finish_kernel applies the group RMSNorm.
+template <int R, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillParams p)
 {
     using Lo = Layout<R>;
@@ -97,11 +100,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
     extern __shared__ __align__(1024) unsigned char smem[];
     cg::cluster_group cluster = cg::this_cluster();
 
-    const int q = (int)cluster.block_rank();            // head within the group
-    const int64_t cid = blockIdx.x / R;                  // (batch row, group)
-    const int64_t bi = cid / p.G;
-    const int g = (int)(cid % p.G);
-    const int h = g * R + q;
+    const int q = (int)cluster.block_rank();            // head within the cluster
+    const int rpg = p.H / p.G;                           // heads per group
+    const int ncl = rpg / R;                             // clusters per group
+    const int64_t cid = blockIdx.x / R;                  // (batch row, group, cluster)
+    const int64_t bi = cid / ((int64_t)p.G * ncl);
+    const int g = (int)((cid / ncl) % p.G);
+    const int h = g * rpg + (int)(cid % ncl) * R + q;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & 127, half = tid >> 7;
     const int64_t HP = p.HP(), GN = p.GN(), Cc = p.Cc();
@@ -110,9 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
     float* mf = reinterpret_cast<float*>(smem + Lo::OFF_MISC);
     float* s_lam = mf + Lo::F_LAM;     // log2-domain inclusive cumsum of delta*A
     float* s_dl = mf + Lo::F_DL;
+    float* s_v = mf + Lo::F_V;         // column factors of the decay mask (see the M build)
     float* s_scan = mf + Lo::F_SCAN;
-    float* s_ssh = mf + Lo::F_SSH;     // [2][128] half sums of g^2
-    float* s_red = mf + Lo::F_RED;     // [R][128] per-head sums of g^2, pushed by every peer
+    float* s_red = mf + Lo::F_RED;     // [R][2][128] per-(head, half) sums of g^2, pushed by every peer
     float* s_cw = mf + Lo::F_CW;       // [SROW][4] conv taps of the staged channels
     float* s_cb = mf + Lo::F_CB;       // [SROW]
     float* s_nw = mf + Lo::F_NW;       // [64] norm weights of this head
@@ -188,11 +193,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
     __nv_bfloat16* gy = (__nv_bfloat16*)p.y;
 
     // issue the raw loads of block k into staging rows 3..3+len-1
-    auto load_block = [&](int64_t k) {
+    auto load_block = [&](int64_t k, int t0i, int nthr) {
         const int64_t t0 = k * kT;
         const int len = (int)min((int64_t)kT, p.L - t0);
         constexpr int CPR = SROW / 8;  // 16-byte chunks per staged row
-        for (int e = tid; e < len * CPR; e += kThreads) {
+        for (int e = t0i; e < len * CPR; e += nthr) {
             const int r = e / CPR, c8 = (e % CPR) * 8;
             const int64_t tok = bi * p.L + t0 + r;
             const __nv_bfloat16* src;
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
         cp_async_commit();
     };
 
-    if (nblk > 0) load_block(0);
+    if (nblk > 0) load_block(0, tid, kThreads);
     float dt_next = 0.0f;
     if (nblk > 0 && tid < kT && tid < p.L)
         dt_next = __bfloat162float(gdt[(bi * p.L + tid) * p.dt_ld + h]);
@@ -227,6 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
         if (tid < kT) { s_lam[tid] = lam; s_dl[tid] = dl; }
         __syncthreads();
         const float lam_end = s_lam[kT - 1];
+        // exp2(lam_i - lam_j) = u_i * v_j with u_i = exp2(lam_i) and v_j = exp2(-lam_j): exact
+        // up to rounding while the factors (and v_j times delta_j) stay normal fp32 numbers.
+        // lam is non-increasing from <= 0, so for a row i with lam_i > -96 every j <= i has
+        // v_j <= 2^96; rows past that decay take exp2 per element. The choice for row i
+        // depends on tokens up to i only, so the result stays causal bit for bit.
+        if (tid < kT) s_v[tid] = (lam > -96.0f) ? ex2(-lam) * dl : 0.0f;
 
         // ---- conv + SiLU of the staged channels: this head's x channels -> x' and x'*w in
         //      shared memory; this CTA's slice of B and C -> every peer's B' and C'.
@@ -294,18 +305,19 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
                 mma_bf16(tmem + kColS, sdesc(aB + kk * 4096, 2048, 128), sdesc(aXW + kk * 2048, 1024, 128), id_s, kk > 0);
             mma_commit(bar0);
         }
-        // raw data of the next block: keep its three halo rows, then start its loads
-        __syncthreads();   // every thread is done reading the staging rows of this block
-        if (k + 1 < nblk) {
-            for (int e = tid; e < 3 * Lo::NV; e += kThreads) {
+        // raw data of the next block: warps 1..7 keep its three halo rows, then start its
+        // loads, while warp 0 issues the MMAs (the conv of every thread finished before the
+        // cluster barrier above, so the staging rows are free)
+        if (k + 1 < nblk && warp > 0) {
+            for (int e = tid - 32; e < 3 * Lo::NV; e += kThreads - 32) {
                 const int r = e % 3, v = e / 3;
                 stage[v * kStageRows + r] = stage[v * kStageRows + kT + r];
             }
-            __syncthreads();
-            load_block(k + 1);
-            if (tid < kT && (k + 1) * kT + tid < p.L)
-                dt_next = __bfloat162float(gdt[(bi * p.L + (k + 1) * kT + tid) * p.dt_ld + h]);
+            asm volatile("bar.sync 1, %0;" ::"n"(kThreads - 32) : "memory");
+            load_block(k + 1, tid - 32, kThreads - 32);
         }
+        if (k + 1 < nblk && tid < kT && (k + 1) * kT + tid < p.L)
+            dt_next = __bfloat162float(gdt[(bi * p.L + (k + 1) * kT + tid) * p.dt_ld + h]);
         // z of this block for the gate, loaded early
         uint4 zr[4];
         {
@@ -331,14 +343,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
             tmem_ld32(tmem + lane_base + kColCB + half * 64 + 32, cb + 32);
             tmem_wait_ld();
             const float li = s_lam[i];
+            const bool fac = li > -96.0f;
+            const float ui = ex2(li);
             unsigned char* sM = smem + OFF_M;
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
                 float m[8];
+                if (fac) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = half * 64 + v * 8 + e;
-                    m[e] = (j <= i) ? cb[v * 8 + e] * ex2(li - s_lam[j]) * s_dl[j] : 0.0f;
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = half * 64 + v * 8 + e;
+                        m[e] = (j <= i) ? cb[v * 8 + e] * (ui * s_v[j]) : 0.0f;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = half * 64 + v * 8 + e;
+                        m[e] = (j <= i) ? cb[v * 8 + e] * ex2(li - s_lam[j]) * s_dl[j] : 0.0f;
+                    }
                 }
                 uint4 u;
                 u.x = pack_bf16x2(m[0], m[1]); u.y = pack_bf16x2(m[2], m[3]);
@@ -402,21 +424,33 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
                     ss = fmaf(gg, gg, ss);
                 }
             }
-            s_ssh[half * 128 + i] = ss;
+            if constexpr (SPLIT) {
+                if (i < len) p.ssp[((bi * p.L + t0 + i) * p.H + h) * 2 + half] = ss;
+            } else {
+#pragma unroll
+                for (int rr = 0; rr < R; ++rr) *cluster.map_shared_rank(s_red + (q * 2 + half) * 128 + i, rr) = ss;
+            }
         }
         fence_before_sync();
-        __syncthreads();
-        if (half == 0) {
-            const float tot = s_ssh[row] + s_ssh[128 + row];
-#pragma unroll
-            for (int rr = 0; rr < R; ++rr) *cluster.map_shared_rank(s_red + q * 128 + row, rr) = tot;
-        }
+        // also orders every peer's MMAs on B' and C' of this block before the next block's
+        // conv writes into them
         cluster.sync();
-        {
+        if constexpr (SPLIT) {
+            if (row < len) {
+                uint4* yo = reinterpret_cast<uint4*>(gy + (bi * p.L + t0 + row) * p.y_ld + (int64_t)h * kP + half * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 u;
+                    u.x = pack_bf16x2(gt[8 * v + 0], gt[8 * v + 1]); u.y = pack_bf16x2(gt[8 * v + 2], gt[8 * v + 3]);
+                    u.z = pack_bf16x2(gt[8 * v + 4], gt[8 * v + 5]); u.w = pack_bf16x2(gt[8 * v + 6], gt[8 * v + 7]);
+                    yo[v] = u;
+                }
+            }
+        } else {
             const int i = row;
             float tot = 0.0f;
 #pragma unroll
-            for (int rr = 0; rr < R; ++rr) tot += s_red[rr * 128 + i];
+            for (int rr = 0; rr < 2 * R; ++rr) tot += s_red[rr * 128 + i];
             const float inv = rsqrtf(tot / (float)(R * kP) + p.eps);
             if (i < len) {
                 uint4* yo = reinterpret_cast<uint4*>(gy + (bi * p.L + t0 + i) * p.y_ld + (int64_t)h * kP + half * 32);
@@ -453,14 +487,45 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_tc_kernel(PrefillPara
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int R>
+// Group RMSNorm of the gated values written by the SPLIT kernel: one warp per
+// (batch row, token, group) sums the 2 * (H/G) partial sums of squares, then rescales the
+// group's H/G * 64 channels in place.
+__global__ void __launch_bounds__(256) norm_finish_kernel(PrefillParams p)
+{
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= p.b * p.L * p.G) return;
+    const int64_t row = w / p.G;
+    const int g = (int)(w % p.G);
+    const int rpg = p.H / p.G, gs = rpg * kP;
+    const float* sp = p.ssp + (row * p.H + (int64_t)g * rpg) * 2;
+    float s = 0.0f;
+    for (int k = lane; k < 2 * rpg; k += 32) s += sp[k];
+    s = warp_sum(s);
+    const float inv = rsqrtf(s / (float)gs + p.eps);
+    __nv_bfloat16* y = (__nv_bfloat16*)p.y + row * p.y_ld + (int64_t)g * gs;
+    const float* nw = p.norm_w + (int64_t)g * gs;
+    for (int c = lane * 8; c < gs; c += 256) {
+        float v[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(y + c), v);
+        uint4 u;
+        u.x = pack_bf16x2(v[0] * inv * nw[c + 0], v[1] * inv * nw[c + 1]);
+        u.y = pack_bf16x2(v[2] * inv * nw[c + 2], v[3] * inv * nw[c + 3]);
+        u.z = pack_bf16x2(v[4] * inv * nw[c + 4], v[5] * inv * nw[c + 5]);
+        u.w = pack_bf16x2(v[6] * inv * nw[c + 6], v[7] * inv * nw[c + 7]);
+        *reinterpret_cast<uint4*>(y + c) = u;
+    }
+}
+
+template <int R, bool SPLIT>
 cudaError_t launch_r(const PrefillParams& p, cudaStream_t st)
 {
     const uint32_t smem = Layout<R>::TOTAL;
-    cudaError_t e = cudaFuncSetAttribute(ssd_prefill_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(ssd_prefill_tc_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.b * p.G * R));
+    cfg.gridDim = dim3((unsigned)(p.b * p.H));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -471,8 +536,18 @@ cudaError_t launch_r(const PrefillParams& p, cudaStream_t st)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    LaunchScope ls("tc_prefill", st);
-    return cudaLaunchKernelEx(&cfg, ssd_prefill_tc_kernel<R>, p);
+    {
+        LaunchScope ls("tc_prefill", st);
+        e = cudaLaunchKernelEx(&cfg, ssd_prefill_tc_kernel<R, SPLIT>, p);
+        if (e != cudaSuccess) return e;
+    }
+    if (SPLIT && p.L > 0) {
+        LaunchScope ls("tc_norm_finish", st);
+        const int64_t warps = p.b * p.L * p.G;
+        norm_finish_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+        e = cudaGetLastError();
+    }
+    return e;
 }
 
 }  // namespace
@@ -480,18 +555,20 @@ cudaError_t launch_r(const PrefillParams& p, cudaStream_t st)
 bool prefill_tc_supported(int act, int P, int N, int H, int G)
 {
     const int r = H / G;
-    return act == 1 && P == kP && N == kN && (r == 2 || r == 4 || r == 8);
+    return act == 1 && P == kP && N == kN && (r == 2 || r == 4 || r == 8 || (r % 8 == 0 && r <= 256));
 }
+
+bool prefill_tc_split(int H, int G) { return H / G > 8; }
 
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t stream)
 {
     if (p.b == 0) return cudaSuccess;
     switch (p.H / p.G) {
-    case 2: return launch_r<2>(p, stream);
-    case 4: return launch_r<4>(p, stream);
-    case 8: return launch_r<8>(p, stream);
+    case 2: return launch_r<2, false>(p, stream);
+    case 4: return launch_r<4, false>(p, stream);
+    case 8: return launch_r<8, false>(p, stream);
     }
-    return cudaErrorInvalidValue;
+    return launch_r<8, true>(p, stream);
 }
 
 }  // namespace ssd
