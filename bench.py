@@ -109,6 +109,10 @@ def kernel_bytes(name, w, batch, seqlen) -> int | None:
         return tok * HP * (4 + 2 * es)
     if name == "decode_step":
         return decode_bytes(w, batch)
+    if name == "tc_prefill":           # the whole prefill in one kernel
+        return path_bytes(w, batch, seqlen, False)
+    if name == "tc_norm_finish":       # gated values read and written, partial sums read
+        return tok * HP * es * 2 + tok * H * 4 * 4
     return None
 
 
@@ -126,7 +130,7 @@ class Clocks:
             try:
                 self.proc = subprocess.Popen(
                     ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                     "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                     "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             except Exception:
                 self.proc = None
 
@@ -320,7 +324,6 @@ def main():
     per_kernel = read_profile(lib)
     lib.ssd_mixer_profile_enable(0)
     barrier()
-    ck = clocks.stop()
     ms_local = e0.elapsed_time(e1) / a.steps
     ms = max_over_ranks(ms_local)
     tok_step = w.batch * (w.seqlen + 1)
@@ -413,6 +416,7 @@ def main():
                   "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                                "frac": ach / hbm, "algorithmic_bytes_per_launch": db, "peak_source": peak_src}}
 
+    ck = clocks.stop()   # sampled over the prefill, end-to-end and decode timed regions
     cpu = None
     if rank == 0 and not a.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, dec, a.cpu_seconds)

@@ -18,7 +18,8 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
         w.status = 0;
         w.xbc = w.delta = w.lam = w.states = w.ypre = w.ssp = 256;
         w.total = 256;
-        if (prefill_tc_split(H, G)) w.total = align256(256 + (size_t)(b * L * H) * 2 * 4);
+        if (prefill_tc_split(H, G))
+            w.total = align256(256 + (size_t)(b * L * H) * (size_t)prefill_tc_partials_per_head() * 4);
         return w;
     }
     const size_t es = act == SSD_BF16 ? 2 : 4;

@@ -36,7 +36,7 @@ struct PrefillParams {
     float* lam;      // [b][H][L] within-chunk inclusive cumsum of delta*A
     float* states;   // [b][nc][H][P][N] chunk states, then states entering each chunk
     float* ypre;     // [b][L][HP] y before the gate and norm
-    float* ssp;      // tensor-core path, groups wider than one cluster: [b][L][H][2] sums of g^2
+    float* ssp;      // tensor-core path, groups wider than one cluster: [b][L][H][parts] sums of g^2
 
     SSD_HD int64_t HP() const { return (int64_t)H * P; }
     SSD_HD int64_t GN() const { return (int64_t)G * N; }
@@ -73,6 +73,7 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
 // every intermediate on chip and needs only the status word of the workspace.
 bool prefill_tc_supported(int act, int P, int N, int H, int G);
 bool prefill_tc_split(int H, int G);   // the group norm is finished by a second kernel
+int prefill_tc_partials_per_head();     // sums of g^2 per (token, head) in split mode
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t stream);
 
 bool prefill_simt_supported(int P, int N);

@@ -49,15 +49,18 @@ def test_static_workspace_prefill_matches_regular_prefill_twice(act):
 
 
 def test_static_workspace_refuses_oversized_problem():
-    w = WORKLOADS["small_bf16"]
-    d = dims_of(w, batch=8, seqlen=4096)
+    # fp32 activations run the CUDA-core path, whose scratch grows with the token count:
+    # 131072 tokens of this shape need more than the fixed array holds
+    w = WORKLOADS["tiny_f32"].with_(batch=1, seqlen=131072)
+    d = dims_of(w)
     assert sm.ssd_mixer_prefill_workspace_size(d) > sm.SSD_MIXER_STATIC_WORKSPACE_BYTES
-    x = torch.zeros(8, 4096, w.d_inner, dtype=torch.bfloat16, device="cuda")
-    bc = torch.zeros(8, 4096, w.ngroups * w.dstate, dtype=torch.bfloat16, device="cuda")
-    dt = torch.zeros(8, 4096, w.nheads, dtype=torch.bfloat16, device="cuda")
+    L, HP, GN = w.seqlen, w.d_inner, w.ngroups * w.dstate
+    x = torch.zeros(1, L, HP, device="cuda")
+    bc = torch.zeros(1, L, GN, device="cuda")
+    dt = torch.zeros(1, L, w.nheads, device="cuda")
     prm = torch.zeros(w.xbc_channels * 4, device="cuda")
-    fs = torch.zeros(8, w.nheads, w.headdim, w.dstate, device="cuda")
-    fc = torch.zeros(8, w.xbc_channels, 3, dtype=torch.bfloat16, device="cuda")
+    fs = torch.zeros(1, w.nheads, w.headdim, w.dstate, device="cuda")
+    fc = torch.zeros(1, w.xbc_channels, 3, device="cuda")
     y = torch.empty_like(x)
     st = sm.ssd_mixer_prefill_static(d, x, x, bc, bc, dt, prm, prm, prm, prm, prm, prm, None, None,
                                      y, fs, fc)
