@@ -19,7 +19,7 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
         w.xbc = w.delta = w.lam = w.states = w.ypre = w.ssp = 256;
         w.total = 256;
         if (prefill_tc_split(H, G))
-            w.total = align256(256 + (size_t)(b * L * H) * (size_t)prefill_tc_partials_per_head() * 4);
+            w.total = align256(256 + (size_t)(b * L * H) * (size_t)prefill_ws_partials_per_head() * 4);
         return w;
     }
     const size_t es = act == SSD_BF16 ? 2 : 4;
@@ -144,7 +144,7 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.ssp = (float*)(ws + wl.ssp);
     cudaStream_t st = (cudaStream_t)stream;
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
-    if ((tc ? ssd::launch_prefill_tc(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
+    if ((tc ? ssd::launch_prefill_ws(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
         return SSD_ERR_CUDA;
     return SSD_OK;
 }

@@ -69,12 +69,14 @@ struct WorkspaceLayout {
 WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
                                          int act);
 
-// Tensor-core path: bf16 activations, P = 64, N = 128, 2, 4 or 8 heads per group. It keeps
-// every intermediate on chip and needs only the status word of the workspace.
+// Tensor-core path (ssd_prefill_ws.cu): bf16 activations, P = 64, N = 128, 2 or a multiple
+// of 4 heads per group. It keeps every intermediate on chip; the workspace holds only the
+// status word, plus per-(token, head) partial sums of squares when the group is wider than
+// one cluster (prefill_tc_split).
 bool prefill_tc_supported(int act, int P, int N, int H, int G);
-bool prefill_tc_split(int H, int G);   // the group norm is finished by a second kernel
-int prefill_tc_partials_per_head();     // sums of g^2 per (token, head) in split mode
-cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t stream);
+bool prefill_tc_split(int H, int G);
+cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream);
+int prefill_ws_partials_per_head();
 
 bool prefill_simt_supported(int P, int N);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t stream);

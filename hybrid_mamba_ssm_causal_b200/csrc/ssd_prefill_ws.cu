@@ -1,0 +1,638 @@
+// ssd_prefill_ws.cu -- warp-specialised, software-pipelined tensor-core prefill of the SSD
+// mixer (bf16 activations, head dim 64, state dim 128).
+//
+// Same arithmetic as one block of the chunked SSD decomposition (Modalities PR #459,
+// ssd.py notes on the chunk-parallel block decomposition) with the state kept on chip:
+// per 128-token block of one head,
+//   lam_i = inclusive sum of delta*A (log2 units), CB = C' B'^T, Ys = C' H^T,
+//   S^T = B'^T (x' w) with w_j = exp(lam_end - lam_j) delta_j,
+//   M_ij = CB_ij exp(lam_i - lam_j) delta_j (j <= i), Yi = M x',
+//   y = Yi + exp(lam_i) Ys + D x',  g = y SiLU(z),  out = g / rms_group(g) * norm_w,
+//   H <- exp(lam_end) H + S.
+// Each CTA owns one head of one batch row; the heads of a cluster share the B/C conv
+// (each CTA convolves a slice and bulk-copies it into every peer) and, when the cluster
+// holds the whole group, the norm's per-token sums of squares (DSMEM).
+//
+// Roles (512 threads):
+//   producer warps 0..7  : raw loads (cp.async), softplus + cumsum, conv + SiLU into the
+//                          operand tiles, the slice exchange, and (thread 0) the MMAs on
+//                          C'B'^T, C'H^T and B'^T(x'w) for block k;
+//   consumer warps 8..15 : for block k-1 meanwhile: the masked decay product M, the state
+//                          update, (thread 256) the MMA M x', the epilogue and the norm.
+// Hand-offs use mbarriers (all waits bounded):
+//   bar0   MMA1-3 of a block done (tensor-core commit)     bar1  MMA4 done
+//   barX   the peers' B'/C' slices of a block have landed (bulk-copy transaction bytes)
+//   barP   producer: softplus/cumsum and x' of a block are in shared memory
+//   barC   consumer: C'B'^T and S^T read from TMEM, H^T of the next block written
+//   barE2  consumer: a block's x' and cumsum buffers are free again (2 slots by parity)
+//   barF2  every CTA of the cluster: its MMA1-3 of a block are done, so its B'/C' may be
+//          overwritten (2 slots, one remote arrival per CTA)
+//   barN2  every CTA of the cluster: its sums of squares of a block are in place
+//          (2 slots, one remote arrival per CTA)
+// Barriers waited two blocks back use two slots, so a waiter never meets a barrier that
+// has moved two phases past the one it expects.
+#include <cooperative_groups.h>
+
+#include "ssd_common.cuh"
+#include "ssd_internal.h"
+#include "ssd_profile.h"
+#include "ssd_tc_util.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace ssd {
+namespace {
+
+using namespace tc;
+
+constexpr int kT = 128;       // tokens per block
+constexpr int kP = 64;        // head dim
+constexpr int kN = 128;       // state dim
+constexpr int kThreads = 512;
+constexpr int kProd = 256;    // producer threads (warps 0..7)
+constexpr int kStageRows = kT + 3;
+constexpr uint32_t kTmemCols = 512;
+constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
+
+// TMEM columns: C'B'^T, Ys (two slots), S^T, Yi
+constexpr uint32_t kColCB = 0, kColYs0 = 128, kColS = 256, kColYi = 320;
+
+// named barriers
+constexpr int kBarProd = 1, kBarCons = 2, kBarScan = 3, kBarHalo = 4;
+
+template <int R>
+struct WsLayout {
+    static constexpr int NS = kN / R;                // B/C channels convolved by one CTA
+    static constexpr int SROW = kP + 2 * NS;
+    static constexpr int NV = SROW / 8;
+    static constexpr uint32_t OFF_C = 0, OFF_B = 32768, OFF_M = 65536, OFF_X = 98304,   // x' [2]
+                              OFF_XW = OFF_X + 2 * 16384, OFF_H = OFF_XW + 16384, OFF_STAGE = OFF_H + 16384;
+    static constexpr uint32_t STAGE_BYTES = (uint32_t)kStageRows * SROW * 2;
+    static constexpr uint32_t OFF_MISC = OFF_STAGE + ((STAGE_BYTES + 127) / 128) * 128;
+    // fp32 arrays: lam, delta, v (2 slots each), scan scratch, sums of squares [2][R][2][128],
+    // conv taps and biases of the staged channels, norm weights
+    static constexpr uint32_t F_LAM = 0, F_DL = 256, F_V = 512, F_SCAN = 768, F_RED = 784,
+                              F_CW = F_RED + 2 * R * 2 * 128, F_CB = F_CW + SROW * 4, F_NW = F_CB + SROW,
+                              F_END = F_NW + kP;
+    static constexpr uint32_t OFF_BAR = OFF_MISC + ((F_END * 4 + 15) / 16) * 16;
+    static constexpr int NBAR = 12;  // bar0 bar1 barX barP barC barE2[2] barF2[2] barN2[2] (+1 slot)
+    static constexpr uint32_t OFF_TSLOT = OFF_BAR + NBAR * 8;
+    static constexpr uint32_t TOTAL = OFF_TSLOT + 16;
+};
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// Arrive on the mbarrier at `mbar_cluster` (a shared::cluster address, possibly a peer's),
+// releasing this thread's prior writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t mbar_cluster)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar_cluster) : "memory");
+}
+
+// Bounded wait whose acquire covers cluster scope (peers' arrivals and DSMEM stores).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t mbar, uint32_t parity, long long limit)
+{
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
+// Inclusive scan over threads 0..127 (warps 0..3; named barrier kBarScan).
+__device__ __forceinline__ float scan128(float v, float* tot)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) tot[wid] = v;
+    named_sync(kBarScan, 128);
+    float off = 0.0f;
+    for (int w = 0; w < wid; ++w) off += tot[w];
+    return v + off;
+}
+
+template <int R, bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillParams p)
+{
+    using Lo = WsLayout<R>;
+    constexpr int NS = Lo::NS, SROW = Lo::SROW;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+
+    const int q = (int)cluster.block_rank();
+    const int rpg = p.H / p.G;
+    const int ncl = rpg / R;
+    const int64_t cid = blockIdx.x / R;
+    const int64_t bi = cid / ((int64_t)p.G * ncl);
+    const int g = (int)((cid / ncl) % p.G);
+    const int h = g * rpg + (int)(cid % ncl) * R + q;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t HP = p.HP(), GN = p.GN(), Cc = p.Cc();
+
+    float* mf = reinterpret_cast<float*>(smem + Lo::OFF_MISC);
+    float* s_lam = mf + Lo::F_LAM;
+    float* s_dl = mf + Lo::F_DL;
+    float* s_v = mf + Lo::F_V;
+    float* s_scan = mf + Lo::F_SCAN;
+    float* s_red = mf + Lo::F_RED;     // [2 slots][R CTAs][2 halves][128 rows]
+    float* s_cw = mf + Lo::F_CW;
+    float* s_cb = mf + Lo::F_CB;
+    float* s_nw = mf + Lo::F_NW;
+    uint4* stage = reinterpret_cast<uint4*>(smem + Lo::OFF_STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lo::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lo::OFF_TSLOT);
+
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t aC = s_base + Lo::OFF_C, aB = s_base + Lo::OFF_B, aM = s_base + Lo::OFF_M;
+    const uint32_t aX = s_base + Lo::OFF_X, aXW = s_base + Lo::OFF_XW, aH = s_base + Lo::OFF_H;
+    const uint32_t bar0 = smem_u32(&bars[0]), bar1 = smem_u32(&bars[1]), barX = smem_u32(&bars[2]);
+    const uint32_t barP = smem_u32(&bars[3]), barC = smem_u32(&bars[4]);
+    const uint32_t barE2 = smem_u32(&bars[5]), barF2 = smem_u32(&bars[7]), barN2 = smem_u32(&bars[9]);
+
+    auto staged_channel = [&](int c) -> int64_t {
+        if (c < kP) return (int64_t)h * kP + c;
+        if (c < kP + NS) return HP + (int64_t)g * kN + (int64_t)q * NS + (c - kP);
+        return HP + GN + (int64_t)g * kN + (int64_t)q * NS + (c - kP - NS);
+    };
+
+    // ---- set-up
+    if (blockIdx.x == 0 && tid == 0) *p.status = 0;
+    for (int c = tid; c < SROW; c += kThreads) {
+        const int64_t ch = staged_channel(c);
+        const float4 w = *reinterpret_cast<const float4*>(p.conv_w + ch * 4);
+        s_cw[c * 4 + 0] = w.x; s_cw[c * 4 + 1] = w.y; s_cw[c * 4 + 2] = w.z; s_cw[c * 4 + 3] = w.w;
+        s_cb[c] = p.conv_b[ch];
+    }
+    if (tid < kP) s_nw[tid] = p.norm_w[(int64_t)h * kP + tid];
+    for (int e = tid; e < 3 * SROW; e += kThreads) {
+        const int k = e / SROW, c = e % SROW;
+        __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
+        if (p.init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(bi * Cc + staged_channel(c)) * 3 + k];
+        reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + k)[c % 8] = v;
+    }
+    if (tid == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar1, 1);
+        mbar_init(barX, 1);
+        mbar_init(barP, 1);
+        mbar_init(barC, 1);
+        mbar_init(barE2, 1);
+        mbar_init(barE2 + 8, 1);
+        mbar_init(barF2, R);
+        mbar_init(barF2 + 8, R);
+        mbar_init(barN2, R);
+        mbar_init(barN2 + 8, R);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+
+    // consumer state: thread (n = row, half) keeps H^T[n][half*32 .. half*32+32) in fp32
+    const bool consumer = tid >= kProd;
+    const int crow = tid & 127, chalf = (tid - kProd) >> 7;   // consumer row and column half
+    float H[32];
+    if (consumer) {
+        const float* h0 = p.init_ssm ? p.init_ssm + (bi * p.H + h) * (int64_t)kP * kN : nullptr;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) H[i] = h0 ? h0[(int64_t)(chalf * 32 + i) * kN + crow] : 0.0f;
+        unsigned char* sH = smem + Lo::OFF_H;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = pack_bf16x2(H[8 * v + 0], H[8 * v + 1]); u.y = pack_bf16x2(H[8 * v + 2], H[8 * v + 3]);
+            u.z = pack_bf16x2(H[8 * v + 4], H[8 * v + 5]); u.w = pack_bf16x2(H[8 * v + 6], H[8 * v + 7]);
+            *reinterpret_cast<uint4*>(sH + canon_off(crow, chalf * 32 + 8 * v, kP)) = u;
+        }
+        fence_async_smem();
+    }
+    fence_before_sync();
+    __syncthreads();
+    cluster.sync();   // every peer's barriers are initialised before any remote arrival or copy
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const float A2 = p.A[h] * 1.4426950408889634f;
+    const float Dh = p.D[h];
+    const float bias = p.dt_bias[h];
+    bool ok = true;
+
+    const int64_t nblk = (p.L + kT - 1) / kT;
+    const __nv_bfloat16* gx = (const __nv_bfloat16*)p.x;
+    const __nv_bfloat16* gB = (const __nv_bfloat16*)p.B;
+    const __nv_bfloat16* gC = (const __nv_bfloat16*)p.C;
+    const __nv_bfloat16* gz = (const __nv_bfloat16*)p.z;
+    const __nv_bfloat16* gdt = (const __nv_bfloat16*)p.dt;
+    __nv_bfloat16* gy = (__nv_bfloat16*)p.y;
+    constexpr uint32_t kSliceBytes = (uint32_t)NS * kT * 2;
+    const uint32_t slice_off = (uint32_t)q * kSliceBytes;
+    auto blen = [&](int64_t k) { return (int)min((int64_t)kT, p.L - k * kT); };
+
+    if (!consumer) {
+        // =========================== producer (warps 0..7) ===========================
+        auto load_block = [&](int64_t k, int t0i, int nthr) {
+            const int64_t t0 = k * kT;
+            const int len = blen(k);
+            constexpr int CPR = SROW / 8;
+            for (int e = t0i; e < len * CPR; e += nthr) {
+                const int r = e / CPR, c8 = (e % CPR) * 8;
+                const int64_t tok = bi * p.L + t0 + r;
+                const __nv_bfloat16* src;
+                if (c8 < kP) src = gx + tok * p.x_ld + (int64_t)h * kP + c8;
+                else if (c8 < kP + NS) src = gB + tok * p.B_ld + (int64_t)g * kN + (int64_t)q * NS + (c8 - kP);
+                else src = gC + tok * p.C_ld + (int64_t)g * kN + (int64_t)q * NS + (c8 - kP - NS);
+                cp_async16(smem_u32(stage + (c8 / 8) * kStageRows + r + 3), src);
+            }
+            cp_async_commit();
+        };
+        float dt_next = 0.0f;
+        if (nblk > 0) {
+            load_block(0, tid, kProd);
+            if (tid < kT && tid < p.L) dt_next = __bfloat162float(gdt[(bi * p.L + tid) * p.dt_ld + h]);
+        }
+        for (int64_t k = 0; k < nblk; ++k) {
+            const int len = blen(k);
+            const int sl = (int)(k & 1);
+            // buffers of this block: x'[sl] and the cumsum slot were last read by the
+            // consumer in block k-2; B'/C'/x'w by this CTA's MMAs of block k-1
+            if (tid == 0) {
+                if (k >= 1 && ok && !mbar_wait_bounded(bar0, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
+                if (k >= 2 && ok && !mbar_wait_bounded(barE2 + 8 * sl, (uint32_t)(((k - 2) >> 1) & 1), kWaitLimit)) ok = false;
+            }
+            cp_async_wait_all();
+            named_sync(kBarProd, kProd);
+            // softplus and cumsum of this block (warps 0..3)
+            if (tid < kT) {
+                float dl = 0.0f, a2 = 0.0f;
+                if (tid < len) {
+                    dl = softplus(dt_next + bias);
+                    a2 = dl * A2;
+                }
+                const float lam = scan128(a2, s_scan);
+                s_lam[sl * kT + tid] = lam;
+                s_dl[sl * kT + tid] = dl;
+                // exp2(lam_i - lam_j) = exp2(lam_i) * exp2(-lam_j) while every factor stays a
+                // normal fp32 number (rows with lam_i > -96); chosen per row from its past only
+                s_v[sl * kT + tid] = (lam > -96.0f) ? ex2(-lam) * dl : 0.0f;
+            }
+            if (tid == 0) mbar_arrive_expect_tx(barX, (uint32_t)(R - 1) * 2 * kSliceBytes);
+            named_sync(kBarProd, kProd);
+            const float* lamb = s_lam + sl * kT;
+            const float* dlb = s_dl + sl * kT;
+            const float lam_end = lamb[kT - 1];
+            // conv + SiLU: x' and x'w of this head, this CTA's slice of B' and C'
+            {
+                unsigned char* sX = smem + Lo::OFF_X + sl * 16384;
+                unsigned char* sXW = smem + Lo::OFF_XW;
+                for (int e = tid; e < Lo::NV * kT; e += kProd) {
+                    const int i = e % kT, v = e / kT;
+                    const int c0 = v * 8;
+                    float o[8];
+                    if (i < len) {
+                        float u[4][8];
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) unpack_bf16x8(stage[v * kStageRows + i + kk], u[kk]);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float* w = s_cw + (c0 + j) * 4;
+                            const float vv = s_cb[c0 + j] + w[0] * u[0][j] + w[1] * u[1][j] + w[2] * u[2][j] + w[3] * u[3][j];
+                            o[j] = silu_fast(vv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) o[j] = 0.0f;
+                    }
+                    uint4 u8;
+                    u8.x = pack_bf16x2(o[0], o[1]); u8.y = pack_bf16x2(o[2], o[3]);
+                    u8.z = pack_bf16x2(o[4], o[5]); u8.w = pack_bf16x2(o[6], o[7]);
+                    if (c0 < kP) {
+                        const float wgt = (i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f;
+                        uint4 uw;
+                        uw.x = pack_bf16x2(o[0] * wgt, o[1] * wgt); uw.y = pack_bf16x2(o[2] * wgt, o[3] * wgt);
+                        uw.z = pack_bf16x2(o[4] * wgt, o[5] * wgt); uw.w = pack_bf16x2(o[6] * wgt, o[7] * wgt);
+                        *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
+                        *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
+                    } else {
+                        const bool isC = c0 >= kP + NS;
+                        const int n0 = q * NS + (isC ? c0 - kP - NS : c0 - kP);
+                        *reinterpret_cast<uint4*>(smem + (isC ? Lo::OFF_C : Lo::OFF_B) + canon_koff(i, n0, kT)) = u8;
+                    }
+                }
+            }
+            fence_async_smem();
+            named_sync(kBarProd, kProd);
+            if (tid == 0) {
+                // the peers' MMAs of block k-1 are done: their B'/C' may take this block's slice
+                if (k >= 1 && ok &&
+                    !mbar_wait_cluster(barF2 + 8 * ((k - 1) & 1), (uint32_t)(((k - 1) >> 1) & 1), kWaitLimit))
+                    ok = false;
+#pragma unroll
+                for (int rr = 0; rr < R; ++rr) {
+                    if (rr == q) continue;
+                    const uint32_t mb = cluster_map(barX, (uint32_t)rr);
+                    bulk_copy_to_peer(cluster_map(aB + slice_off, (uint32_t)rr), aB + slice_off, kSliceBytes, mb);
+                    bulk_copy_to_peer(cluster_map(aC + slice_off, (uint32_t)rr), aC + slice_off, kSliceBytes, mb);
+                }
+                if (ok && !mbar_wait_bounded(barX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
+                // the consumer has read C'B'^T and S^T of block k-1 and written H^T for this block
+                if (k >= 1 && ok && !mbar_wait_bounded(barC, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
+                mbar_arrive_local(barP);   // this block's cumsum and x' are in place
+                fence_after_sync();
+                const uint32_t id_cb = idesc_bf16(128, 128, 0, 0);
+                const uint32_t id_ys = idesc_bf16(128, 64, 0, 1);
+                const uint32_t id_s = idesc_bf16(128, 64, 1, 1);
+                const uint32_t colYs = kColYs0 + 64 * (uint32_t)sl;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + kColCB, sdesc(aC + kk * 4096, 2048, 128), sdesc(aB + kk * 4096, 2048, 128), id_cb, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + colYs, sdesc(aC + kk * 4096, 2048, 128), sdesc(aH + kk * 2048, 1024, 128), id_ys, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + kColS, sdesc(aB + kk * 256, 128, 2048), sdesc(aXW + kk * 2048, 1024, 128), id_s, kk > 0);
+                mma_commit(bar0);
+            }
+            // raw rows of the next block (warps 1..7): halo, then the loads; dt of the next block
+            if (k + 1 < nblk && warp > 0) {
+                for (int e = tid - 32; e < 3 * Lo::NV; e += kProd - 32) {
+                    const int r = e % 3, v = e / 3;
+                    stage[v * kStageRows + r] = stage[v * kStageRows + kT + r];
+                }
+                named_sync(kBarHalo, kProd - 32);
+                load_block(k + 1, tid - 32, kProd - 32);
+            }
+            if (k + 1 < nblk && tid < kT && (k + 1) * kT + tid < p.L)
+                dt_next = __bfloat162float(gdt[(bi * p.L + (k + 1) * kT + tid) * p.dt_ld + h]);
+        }
+        // final conv state: the last three raw inputs of the staged channels
+        const int len_last = nblk > 0 ? blen(nblk - 1) : 0;
+        named_sync(kBarProd, kProd);
+        for (int e = tid; e < 3 * SROW; e += kProd) {
+            const int kk = e / SROW, c = e % SROW;
+            ((__nv_bfloat16*)p.final_conv)[(bi * Cc + staged_channel(c)) * 3 + kk] =
+                reinterpret_cast<const __nv_bfloat16*>(stage + (c / 8) * kStageRows + len_last + kk)[c % 8];
+        }
+    } else {
+        // =========================== consumer (warps 8..15) ===========================
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        for (int64_t k = 0; k < nblk; ++k) {
+            const int64_t t0 = k * kT;
+            const int len = blen(k);
+            const int sl = (int)(k & 1);
+            const uint32_t par = (uint32_t)(k & 1);
+            // z of this block for the gate
+            uint4 zr[4];
+            if (crow < len) {
+                const uint4* zs = reinterpret_cast<const uint4*>(gz + (bi * p.L + t0 + crow) * p.z_ld + (int64_t)h * kP + chalf * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) zr[v] = zs[v];
+            } else {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) zr[v] = make_uint4(0, 0, 0, 0);
+            }
+            if (ok && !mbar_wait_bounded(barP, par, kWaitLimit)) ok = false;
+            if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
+            fence_after_sync();
+            // this CTA's MMAs on B'/C' of block k are done: tell every peer
+            if (tid == kProd) {
+#pragma unroll
+                for (int rr = 0; rr < R; ++rr) mbar_arrive_remote(cluster_map(barF2 + 8 * sl, (uint32_t)rr));
+            }
+            const float* lamb = s_lam + sl * kT;
+            const float* dlb = s_dl + sl * kT;
+            const float* vb = s_v + sl * kT;
+            const float lam_end = lamb[kT - 1];
+            // masked, decayed M (row crow, columns chalf*64 .. +64), bf16, K-major
+            {
+                const int i = crow;
+                const float li = lamb[i];
+                const bool fac = li > -96.0f;
+                const float ui = ex2(li);
+                unsigned char* sM = smem + Lo::OFF_M;
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    float cb[32];
+                    tmem_ld32(tmem + lane_base + kColCB + chalf * 64 + part * 32, cb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        float m[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = chalf * 64 + part * 32 + v * 8 + e;
+                            const float dec = fac ? ui * vb[j] : ex2(li - lamb[j]) * dlb[j];
+                            m[e] = (j <= i) ? cb[v * 8 + e] * dec : 0.0f;
+                        }
+                        uint4 u;
+                        u.x = pack_bf16x2(m[0], m[1]); u.y = pack_bf16x2(m[2], m[3]);
+                        u.z = pack_bf16x2(m[4], m[5]); u.w = pack_bf16x2(m[6], m[7]);
+                        *reinterpret_cast<uint4*>(sM + canon_off(i, chalf * 64 + part * 32 + v * 8, kT)) = u;
+                    }
+                }
+            }
+            // state update H <- exp(lam_end) H + S and its bf16 copy for the next block
+            {
+                float s_[32];
+                tmem_ld32(tmem + lane_base + kColS + chalf * 32, s_);
+                tmem_wait_ld();
+                const float aend = ex2(lam_end);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) H[i] = fmaf(aend, H[i], s_[i]);
+                unsigned char* sH = smem + Lo::OFF_H;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 u;
+                    u.x = pack_bf16x2(H[8 * v + 0], H[8 * v + 1]); u.y = pack_bf16x2(H[8 * v + 2], H[8 * v + 3]);
+                    u.z = pack_bf16x2(H[8 * v + 4], H[8 * v + 5]); u.w = pack_bf16x2(H[8 * v + 6], H[8 * v + 7]);
+                    *reinterpret_cast<uint4*>(sH + canon_off(crow, chalf * 32 + 8 * v, kP)) = u;
+                }
+            }
+            fence_async_smem();
+            fence_before_sync();
+            named_sync(kBarCons, kThreads - kProd);
+            if (tid == kProd) {
+                mbar_arrive_local(barC);   // C'B'^T and S^T read, H^T of block k+1 written
+                fence_after_sync();
+                const uint32_t id_yi = idesc_bf16(128, 64, 0, 1);
+                const uint32_t aXs = aX + 16384 * (uint32_t)sl;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + kColYi, sdesc(aM + kk * 256, 128, 2048), sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
+                mma_commit(bar1);
+            }
+            if (ok && !mbar_wait_bounded(bar1, par, kWaitLimit)) ok = false;
+            fence_after_sync();
+            // epilogue: y = Yi + exp(lam_i) Ys + D x', gate
+            float gt[32];
+            {
+                const int i = crow;
+                float yi[32], ys[32];
+                tmem_ld32(tmem + lane_base + kColYi + chalf * 32, yi);
+                tmem_ld32(tmem + lane_base + kColYs0 + 64 * sl + chalf * 32, ys);
+                tmem_wait_ld();
+                const float el = ex2(lamb[i]);
+                const unsigned char* sX = smem + Lo::OFF_X + sl * 16384;
+                float ss = 0.0f;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    float xv[8], zv[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sX + canon_off(i, chalf * 32 + 8 * v, kP)), xv);
+                    unpack_bf16x8(zr[v], zv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int c = 8 * v + e;
+                        const float y = fmaf(el, ys[c], yi[c]) + Dh * xv[e];
+                        const float gg = y * silu_fast(zv[e]);
+                        gt[c] = gg;
+                        ss = fmaf(gg, gg, ss);
+                    }
+                }
+                if constexpr (SPLIT) {
+                    if (i < len) p.ssp[((bi * p.L + t0 + i) * p.H + h) * 2 + chalf] = ss;
+                } else {
+#pragma unroll
+                    for (int rr = 0; rr < R; ++rr)
+                        *cluster.map_shared_rank(s_red + ((sl * R + q) * 2 + chalf) * 128 + i, rr) = ss;
+                }
+            }
+            fence_before_sync();
+            named_sync(kBarCons, kThreads - kProd);
+            if (tid == kProd) {
+                mbar_arrive_local(barE2 + 8 * sl);   // x'[sl] and the cumsum slot are free
+                if constexpr (!SPLIT) {
+#pragma unroll
+                    for (int rr = 0; rr < R; ++rr) mbar_arrive_remote(cluster_map(barN2 + 8 * sl, (uint32_t)rr));
+                }
+            }
+            float scale = 1.0f;
+            if constexpr (!SPLIT) {
+                if (ok && !mbar_wait_cluster(barN2 + 8 * sl, (uint32_t)((k >> 1) & 1), kWaitLimit)) ok = false;
+                float tot = 0.0f;
+#pragma unroll
+                for (int rr = 0; rr < 2 * R; ++rr) tot += s_red[(sl * R * 2 + rr) * 128 + crow];
+                scale = rsqrtf(tot / (float)(R * kP) + p.eps);
+            }
+            if (crow < len) {
+                uint4* yo = reinterpret_cast<uint4*>(gy + (bi * p.L + t0 + crow) * p.y_ld + (int64_t)h * kP + chalf * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o[e] = SPLIT ? gt[8 * v + e] : gt[8 * v + e] * scale * s_nw[chalf * 32 + 8 * v + e];
+                    uint4 u;
+                    u.x = pack_bf16x2(o[0], o[1]); u.y = pack_bf16x2(o[2], o[3]);
+                    u.z = pack_bf16x2(o[4], o[5]); u.w = pack_bf16x2(o[6], o[7]);
+                    yo[v] = u;
+                }
+            }
+        }
+        // final SSM state of this head
+        float* fs = p.final_ssm + (bi * p.H + h) * (int64_t)kP * kN;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) fs[(int64_t)(chalf * 32 + i) * kN + crow] = H[i];
+    }
+
+    if (!ok) atomicExch(p.status, 1);
+    fence_before_sync();
+    __syncthreads();
+    cluster.sync();   // no peer still copies into or arrives on this CTA's shared memory
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Group RMSNorm of the gated values written by the SPLIT kernel (2 partial sums per head).
+__global__ void __launch_bounds__(256) ws_norm_finish_kernel(PrefillParams p)
+{
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= p.b * p.L * p.G) return;
+    const int64_t row = w / p.G;
+    const int g = (int)(w % p.G);
+    const int rpg = p.H / p.G, gs = rpg * kP;
+    const float* sp = p.ssp + (row * p.H + (int64_t)g * rpg) * 2;
+    float s = 0.0f;
+    for (int k = lane; k < 2 * rpg; k += 32) s += sp[k];
+    s = warp_sum(s);
+    const float inv = rsqrtf(s / (float)gs + p.eps);
+    __nv_bfloat16* y = (__nv_bfloat16*)p.y + row * p.y_ld + (int64_t)g * gs;
+    const float* nw = p.norm_w + (int64_t)g * gs;
+    for (int c = lane * 8; c < gs; c += 256) {
+        float v[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(y + c), v);
+        uint4 u;
+        u.x = pack_bf16x2(v[0] * inv * nw[c + 0], v[1] * inv * nw[c + 1]);
+        u.y = pack_bf16x2(v[2] * inv * nw[c + 2], v[3] * inv * nw[c + 3]);
+        u.z = pack_bf16x2(v[4] * inv * nw[c + 4], v[5] * inv * nw[c + 5]);
+        u.w = pack_bf16x2(v[6] * inv * nw[c + 6], v[7] * inv * nw[c + 7]);
+        *reinterpret_cast<uint4*>(y + c) = u;
+    }
+}
+
+template <int R, bool SPLIT>
+cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
+{
+    using Lo = WsLayout<R>;
+    cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Lo::TOTAL);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.b * p.H));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Lo::TOTAL;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = R;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+        LaunchScope ls("tc_prefill", st);
+        e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT>, p);
+        if (e != cudaSuccess) return e;
+    }
+    if (SPLIT && p.L > 0) {
+        LaunchScope ls("tc_norm_finish", st);
+        const int64_t warps = p.b * p.L * p.G;
+        ws_norm_finish_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace
+
+// Groups of 2 or 4 heads: one cluster per group (fused norm); wider groups: clusters of 4
+// heads and the norm finished by ws_norm_finish_kernel.
+cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream)
+{
+    if (p.b == 0) return cudaSuccess;
+    switch (p.H / p.G) {
+    case 2: return launch_ws<2, false>(p, stream);
+    case 4: return launch_ws<4, false>(p, stream);
+    }
+    return launch_ws<4, true>(p, stream);
+}
+
+int prefill_ws_partials_per_head() { return 2; }
+
+bool prefill_tc_supported(int act, int P, int N, int H, int G)
+{
+    const int r = H / G;
+    return act == 1 && P == kP && N == kN && (r == 2 || (r % 4 == 0 && r <= 256));
+}
+
+bool prefill_tc_split(int H, int G) { return H / G > 4; }
+
+}  // namespace ssd

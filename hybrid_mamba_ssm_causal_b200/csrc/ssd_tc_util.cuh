@@ -54,6 +54,12 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
         : "memory");
 }
 
+// Plain arrival on a local mbarrier (release at CTA scope).
+__device__ __forceinline__ void mbar_arrive_local(uint32_t mbar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
 // Arrive on an mbarrier and raise its expected transaction count by `bytes`.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes)
 {
