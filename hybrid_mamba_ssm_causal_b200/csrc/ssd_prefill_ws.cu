@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     for (int c = tid; c < SROW; c += kThreads) {
         const int64_t ch = staged_channel(c);
         const float4 w = *reinterpret_cast<const float4*>(p.conv_w + ch * 4);
-        s_cw[c * 4 + 0] = w.x; s_cw[c * 4 + 1] = w.y; s_cw[c * 4 + 2] = w.z; s_cw[c * 4 + 3] = w.w;
+        float* cw = s_cw + (c / 2) * 8 + (c % 2);   // taps of channel pairs: [pair][tap][2]
+        cw[0] = w.x; cw[2] = w.y; cw[4] = w.z; cw[6] = w.w;
         s_cb[c] = p.conv_b[ch];
     }
     if (tid < kP) s_nw[tid] = p.norm_w[(int64_t)h * kP + tid];
@@ -293,38 +294,67 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             {
                 unsigned char* sX = smem + Lo::OFF_X + sl * 16384;
                 unsigned char* sXW = smem + Lo::OFF_XW;
-                for (int e = tid; e < Lo::NV * kT; e += kProd) {
-                    const int i = e % kT, v = e / kT;
+                // Work split: 16 threads per 8-channel vector v, each taking rows i = t%16 + 16m,
+                // so a warp covers 16 consecutive rows of 2 vectors (conflict-free staged reads
+                // and canonical stores) and a thread keeps its vector's taps in registers.
+                constexpr int kPasses = (Lo::NV + 15) / 16;
+                for (int pass = 0; pass < kPasses; ++pass) {
+                    const int v = pass * 16 + tid / 16;
+                    if (v >= Lo::NV) break;
                     const int c0 = v * 8;
-                    float o[8];
-                    if (i < len) {
-                        float u[4][8];
+                    float2 wr[4][4], br[4];
+                    {
+                        const float2* cw2 = reinterpret_cast<const float2*>(s_cw) + (c0 / 2) * 4;
+                        const float2* cb2 = reinterpret_cast<const float2*>(s_cb) + c0 / 2;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) unpack_bf16x8(stage[v * kStageRows + i + kk], u[kk]);
+                        for (int j = 0; j < 4; ++j) {
+                            br[j] = cb2[j];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float* w = s_cw + (c0 + j) * 4;
-                            const float vv = s_cb[c0 + j] + w[0] * u[0][j] + w[1] * u[1][j] + w[2] * u[2][j] + w[3] * u[3][j];
-                            o[j] = silu_fast(vv);
+                            for (int kk = 0; kk < 4; ++kk) wr[j][kk] = cw2[j * 4 + kk];
                         }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) o[j] = 0.0f;
                     }
-                    uint4 u8;
-                    u8.x = pack_bf16x2(o[0], o[1]); u8.y = pack_bf16x2(o[2], o[3]);
-                    u8.z = pack_bf16x2(o[4], o[5]); u8.w = pack_bf16x2(o[6], o[7]);
-                    if (c0 < kP) {
-                        const float wgt = (i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f;
-                        uint4 uw;
-                        uw.x = pack_bf16x2(o[0] * wgt, o[1] * wgt); uw.y = pack_bf16x2(o[2] * wgt, o[3] * wgt);
-                        uw.z = pack_bf16x2(o[4] * wgt, o[5] * wgt); uw.w = pack_bf16x2(o[6] * wgt, o[7] * wgt);
-                        *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
-                        *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
-                    } else {
-                        const bool isC = c0 >= kP + NS;
-                        const int n0 = q * NS + (isC ? c0 - kP - NS : c0 - kP);
-                        *reinterpret_cast<uint4*>(smem + (isC ? Lo::OFF_C : Lo::OFF_B) + canon_koff(i, n0, kT)) = u8;
+                    const bool is_x = c0 < kP;
+                    const bool isC = c0 >= kP + NS;
+                    const int n0 = q * NS + (isC ? c0 - kP - NS : c0 - kP);
+                    unsigned char* dstBC = smem + (isC ? Lo::OFF_C : Lo::OFF_B);
+#pragma unroll 1
+                    for (int m = 0; m < 8; m += 2) {
+                        int ii[2];
+                        uint4 raw[2][4];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            ii[u] = (tid % 16) + 16 * (m + u);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) raw[u][kk] = stage[v * kStageRows + ii[u] + kk];
+                        }
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int i = ii[u];
+                            float2 o[4];
+                            if (i < len) {
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {   // channel pair (c0 + 2j, c0 + 2j + 1)
+                                    float2 vv = fma2(wr[j][0], bf2_to_f2((&raw[u][0].x)[j]), br[j]);
+                                    vv = fma2(wr[j][1], bf2_to_f2((&raw[u][1].x)[j]), vv);
+                                    vv = fma2(wr[j][2], bf2_to_f2((&raw[u][2].x)[j]), vv);
+                                    vv = fma2(wr[j][3], bf2_to_f2((&raw[u][3].x)[j]), vv);
+                                    o[j] = silu2(vv);
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) o[j] = make_float2(0.0f, 0.0f);
+                            }
+                            const uint4 u8 = make_uint4(pack_f2(o[0]), pack_f2(o[1]), pack_f2(o[2]), pack_f2(o[3]));
+                            if (is_x) {
+                                const float2 wgt = splat2((i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f);
+                                const uint4 uw = make_uint4(pack_f2(mul2(o[0], wgt)), pack_f2(mul2(o[1], wgt)),
+                                                            pack_f2(mul2(o[2], wgt)), pack_f2(mul2(o[3], wgt)));
+                                *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
+                                *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
+                            } else {
+                                *reinterpret_cast<uint4*>(dstBC + canon_koff(i, n0, kT)) = u8;
+                            }
+                        }
                     }
                 }
             }
@@ -419,23 +449,39 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 const bool fac = li > -96.0f;
                 const float ui = ex2(li);
                 unsigned char* sM = smem + Lo::OFF_M;
+                float cbf[64];
+                tmem_ld32(tmem + lane_base + kColCB + chalf * 64, cbf);
+                tmem_ld32(tmem + lane_base + kColCB + chalf * 64 + 32, cbf + 32);
+                tmem_wait_ld();
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
-                    float cb[32];
-                    tmem_ld32(tmem + lane_base + kColCB + chalf * 64 + part * 32, cb);
-                    tmem_wait_ld();
+                    const float* cb = cbf + part * 32;
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
-                        float m[8];
+                        const int j0 = chalf * 64 + part * 32 + v * 8;
+                        uint32_t w[4];
+                        if (j0 > i) {                 // above the diagonal: all zero
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = chalf * 64 + part * 32 + v * 8 + e;
-                            const float dec = fac ? ui * vb[j] : ex2(li - lamb[j]) * dlb[j];
-                            m[e] = (j <= i) ? cb[v * 8 + e] * dec : 0.0f;
+                            for (int e = 0; e < 4; ++e) w[e] = 0u;
+                        } else if (fac) {
+                            const float2* v2 = reinterpret_cast<const float2*>(vb + j0);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float2 m = mul2(make_float2(cb[v * 8 + 2 * e], cb[v * 8 + 2 * e + 1]), mul2(splat2(ui), v2[e]));
+                                if (j0 + 2 * e > i) m.x = 0.0f;
+                                if (j0 + 2 * e + 1 > i) m.y = 0.0f;
+                                w[e] = pack_f2(m);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = j0 + 2 * e;
+                                const float mx = (j <= i) ? cb[v * 8 + 2 * e] * ex2(li - lamb[j]) * dlb[j] : 0.0f;
+                                const float my = (j + 1 <= i) ? cb[v * 8 + 2 * e + 1] * ex2(li - lamb[j + 1]) * dlb[j + 1] : 0.0f;
+                                w[e] = pack_bf16x2(mx, my);
+                            }
                         }
-                        uint4 u;
-                        u.x = pack_bf16x2(m[0], m[1]); u.y = pack_bf16x2(m[2], m[3]);
-                        u.z = pack_bf16x2(m[4], m[5]); u.w = pack_bf16x2(m[6], m[7]);
+                        const uint4 u = make_uint4(w[0], w[1], w[2], w[3]);
                         *reinterpret_cast<uint4*>(sM + canon_off(i, chalf * 64 + part * 32 + v * 8, kT)) = u;
                     }
                 }
@@ -445,9 +491,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 float s_[32];
                 tmem_ld32(tmem + lane_base + kColS + chalf * 32, s_);
                 tmem_wait_ld();
-                const float aend = ex2(lam_end);
+                const float2 aend = splat2(ex2(lam_end));
 #pragma unroll
-                for (int i = 0; i < 32; ++i) H[i] = fmaf(aend, H[i], s_[i]);
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 hv = fma2(aend, make_float2(H[i], H[i + 1]), make_float2(s_[i], s_[i + 1]));
+                    H[i] = hv.x;
+                    H[i + 1] = hv.y;
+                }
                 unsigned char* sH = smem + Lo::OFF_H;
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
@@ -480,23 +530,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 tmem_ld32(tmem + lane_base + kColYi + chalf * 32, yi);
                 tmem_ld32(tmem + lane_base + kColYs0 + 64 * sl + chalf * 32, ys);
                 tmem_wait_ld();
-                const float el = ex2(lamb[i]);
+                const float2 el = splat2(ex2(lamb[i])), d2 = splat2(Dh);
                 const unsigned char* sX = smem + Lo::OFF_X + sl * 16384;
-                float ss = 0.0f;
+                float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    float xv[8], zv[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sX + canon_off(i, chalf * 32 + 8 * v, kP)), xv);
-                    unpack_bf16x8(zr[v], zv);
+                    const uint4 xw = *reinterpret_cast<const uint4*>(sX + canon_off(i, chalf * 32 + 8 * v, kP));
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int c = 8 * v + e;
-                        const float y = fmaf(el, ys[c], yi[c]) + Dh * xv[e];
-                        const float gg = y * silu_fast(zv[e]);
-                        gt[c] = gg;
-                        ss = fmaf(gg, gg, ss);
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 8 * v + 2 * e;
+                        float2 y = fma2(el, make_float2(ys[c], ys[c + 1]), make_float2(yi[c], yi[c + 1]));
+                        y = fma2(d2, bf2_to_f2((&xw.x)[e]), y);
+                        const float2 gg = mul2(y, silu2(bf2_to_f2((&zr[v].x)[e])));
+                        gt[c] = gg.x;
+                        gt[c + 1] = gg.y;
+                        ss2 = fma2(gg, gg, ss2);
                     }
                 }
+                const float ss = ss2.x + ss2.y;
                 if constexpr (SPLIT) {
                     if (i < len) p.ssp[((bi * p.L + t0 + i) * p.H + h) * 2 + chalf] = ss;
                 } else {
@@ -524,16 +575,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             }
             if (crow < len) {
                 uint4* yo = reinterpret_cast<uint4*>(gy + (bi * p.L + t0 + crow) * p.y_ld + (int64_t)h * kP + chalf * 32);
+                const float2* nw2 = reinterpret_cast<const float2*>(s_nw + chalf * 32);
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    float o[8];
+                    uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o[e] = SPLIT ? gt[8 * v + e] : gt[8 * v + e] * scale * s_nw[chalf * 32 + 8 * v + e];
-                    uint4 u;
-                    u.x = pack_bf16x2(o[0], o[1]); u.y = pack_bf16x2(o[2], o[3]);
-                    u.z = pack_bf16x2(o[4], o[5]); u.w = pack_bf16x2(o[6], o[7]);
-                    yo[v] = u;
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 gg = make_float2(gt[8 * v + 2 * e], gt[8 * v + 2 * e + 1]);
+                        w[e] = pack_f2(SPLIT ? gg : mul2(mul2(gg, splat2(scale)), nw2[4 * v + e]));
+                    }
+                    yo[v] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
         }

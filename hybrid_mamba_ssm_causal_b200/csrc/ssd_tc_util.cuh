@@ -225,6 +225,46 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// Packed pairs of fp32 (sm_100 f32x2 instructions: one issue, two lanes, each rounded
+// to nearest like its scalar counterpart).
+__device__ __forceinline__ unsigned long long f2u(float2 v)
+{
+    return ((unsigned long long)__float_as_uint(v.y) << 32) | __float_as_uint(v.x);
+}
+__device__ __forceinline__ float2 u2f(unsigned long long r)
+{
+    return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
+    return u2f(r);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2u(a)), "l"(f2u(b)));
+    return u2f(r);
+}
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 silu2(float2 v)
+{
+    const float2 h = mul2(v, splat2(0.5f));
+    const float2 t = make_float2(tanh_approx(h.x), tanh_approx(h.y));
+    return mul2(v, fma2(t, splat2(0.5f), splat2(0.5f)));
+}
+// two bf16 in one 32-bit word -> float2 (low half first)
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w)
+{
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t pack_f2(float2 v)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
