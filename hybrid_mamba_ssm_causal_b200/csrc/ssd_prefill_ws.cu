@@ -27,8 +27,8 @@
 //   barE2  consumer: a block's x' and cumsum buffers are free again (2 slots by parity)
 //   barF2  every CTA of the cluster: its MMA1-3 of a block are done, so its B'/C' may be
 //          overwritten (2 slots, one remote arrival per CTA)
-//   barN2  every CTA of the cluster: its sums of squares of a block are in place
-//          (2 slots, one remote arrival per CTA)
+//   barN2  the sums of squares of a block from every CTA of the cluster have landed
+//          (st.async transaction bytes; 2 slots)
 // Barriers waited two blocks back use two slots, so a waiter never meets a barrier that
 // has moved two phases past the one it expects.
 #include <cooperative_groups.h>
@@ -82,11 +82,21 @@ struct WsLayout {
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-// Arrive on the mbarrier at `mbar_cluster` (a shared::cluster address, possibly a peer's),
-// releasing this thread's prior writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t mbar_cluster)
+// Arrive on the mbarrier at `mbar_cluster` (a shared::cluster address, possibly a peer's)
+// without ordering this thread's earlier memory operations: used to say that this CTA's
+// MMAs, already seen complete, no longer read its B'/C' tiles.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t mbar_cluster)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar_cluster) : "memory");
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar_cluster) : "memory");
+}
+
+// 4-byte store into a peer's shared memory that completes 4 transaction bytes on the
+// peer's mbarrier (both shared::cluster addresses).
+__device__ __forceinline__ void st_async_f32(uint32_t dst_cluster, float v, uint32_t mbar_cluster)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst_cluster),
+                 "r"(__float_as_uint(v)), "r"(mbar_cluster)
+                 : "memory");
 }
 
 // Bounded wait whose acquire covers cluster scope (peers' arrivals and DSMEM stores).
@@ -193,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         mbar_init(barE2 + 8, 1);
         mbar_init(barF2, R);
         mbar_init(barF2 + 8, R);
-        mbar_init(barN2, R);
-        mbar_init(barN2 + 8, R);
+        mbar_init(barN2, 1);
+        mbar_init(barN2 + 8, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -433,10 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             if (ok && !mbar_wait_bounded(barP, par, kWaitLimit)) ok = false;
             if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
             fence_after_sync();
-            // this CTA's MMAs on B'/C' of block k are done: tell every peer
+            // this CTA's MMAs on B'/C' of block k are done: tell every peer; and expect the
+            // peers' sums of squares of block k (2 floats per row from every CTA)
             if (tid == kProd) {
 #pragma unroll
-                for (int rr = 0; rr < R; ++rr) mbar_arrive_remote(cluster_map(barF2 + 8 * sl, (uint32_t)rr));
+                for (int rr = 0; rr < R; ++rr) mbar_arrive_remote_relaxed(cluster_map(barF2 + 8 * sl, (uint32_t)rr));
+                if constexpr (!SPLIT) mbar_arrive_expect_tx(barN2 + 8 * sl, (uint32_t)(R * 2 * 128 * 4));
             }
             const float* lamb = s_lam + sl * kT;
             const float* dlb = s_dl + sl * kT;
@@ -551,20 +563,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 if constexpr (SPLIT) {
                     if (i < len) p.ssp[((bi * p.L + t0 + i) * p.H + h) * 2 + chalf] = ss;
                 } else {
+                    const uint32_t dst = smem_u32(s_red + ((sl * R + q) * 2 + chalf) * 128 + i);
 #pragma unroll
                     for (int rr = 0; rr < R; ++rr)
-                        *cluster.map_shared_rank(s_red + ((sl * R + q) * 2 + chalf) * 128 + i, rr) = ss;
+                        st_async_f32(cluster_map(dst, (uint32_t)rr), ss, cluster_map(barN2 + 8 * sl, (uint32_t)rr));
                 }
             }
             fence_before_sync();
             named_sync(kBarCons, kThreads - kProd);
-            if (tid == kProd) {
-                mbar_arrive_local(barE2 + 8 * sl);   // x'[sl] and the cumsum slot are free
-                if constexpr (!SPLIT) {
-#pragma unroll
-                    for (int rr = 0; rr < R; ++rr) mbar_arrive_remote(cluster_map(barN2 + 8 * sl, (uint32_t)rr));
-                }
-            }
+            if (tid == kProd) mbar_arrive_local(barE2 + 8 * sl);   // x'[sl] and the cumsum slot are free
             float scale = 1.0f;
             if constexpr (!SPLIT) {
                 if (ok && !mbar_wait_cluster(barN2 + 8 * sl, (uint32_t)((k >> 1) & 1), kWaitLimit)) ok = false;
