@@ -26,12 +26,19 @@
 //   barC   consumer: C'B'^T and S^T read from TMEM, H^T of the next block written
 //   barE2  consumer: a block's x' and cumsum buffers are free again (2 slots by parity)
 //   barF2  every CTA of the cluster: its MMA1-3 of a block are done, so its B'/C' may be
-//          overwritten (2 slots, one remote arrival per CTA)
-//   barN2  the sums of squares of a block from every CTA of the cluster have landed
-//          (st.async transaction bytes; 2 slots)
+//          overwritten (2 slots; one arrival per CTA, multicast by its tensor-core commit)
+//   barN3  the sums of squares of a block from every CTA of the cluster have landed
+//          (st.async transaction bytes; 3 slots)
 // Barriers waited two blocks back use two slots, so a waiter never meets a barrier that
-// has moved two phases past the one it expects.
+// has moved two phases past the one it expects. The group norm of block k is finished one
+// block late (its gated values wait in TMEM), while the MMA of block k+1 runs; a peer can
+// be at most two blocks ahead of that finish, hence three slots for the sums of squares.
 #include <cooperative_groups.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <type_traits>
 
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
@@ -50,15 +57,17 @@ constexpr int kP = 64;        // head dim
 constexpr int kN = 128;       // state dim
 constexpr int kThreads = 512;
 constexpr int kProd = 256;    // producer threads (warps 0..7)
-constexpr int kStageRows = kT + 3;
+// Raw staging of one 8-channel vector: rows 5..7 hold the three tokens before the block
+// (the conv halo), rows 8..135 the block's tokens (one TMA box, 128-byte aligned).
+constexpr int kStageRows = 136, kStageTok = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
 
-// TMEM columns: C'B'^T, Ys (two slots), S^T, Yi
-constexpr uint32_t kColCB = 0, kColYs0 = 128, kColS = 256, kColYi = 320;
+// TMEM columns: C'B'^T, Ys (two slots), S^T, Yi, the gated values of a block awaiting its norm
+constexpr uint32_t kColCB = 0, kColYs0 = 128, kColS = 256, kColYi = 320, kColG = 384;
 
 // named barriers
-constexpr int kBarProd = 1, kBarCons = 2, kBarScan = 3, kBarHalo = 4;
+constexpr int kBarProd = 1, kBarCons = 2, kBarScan = 3, kBarHalo = 4, kBarHaloX = 5;
 
 template <int R>
 struct WsLayout {
@@ -67,28 +76,20 @@ struct WsLayout {
     static constexpr int NV = SROW / 8;
     static constexpr uint32_t OFF_C = 0, OFF_B = 32768, OFF_M = 65536, OFF_X = 98304,   // x' [2]
                               OFF_XW = OFF_X + 2 * 16384, OFF_H = OFF_XW + 16384, OFF_STAGE = OFF_H + 16384;
-    static constexpr uint32_t STAGE_BYTES = (uint32_t)kStageRows * SROW * 2;
+    static constexpr uint32_t STAGE_BYTES = (uint32_t)kStageRows * SROW * 2;   // SROW/8 vectors
     static constexpr uint32_t OFF_MISC = OFF_STAGE + ((STAGE_BYTES + 127) / 128) * 128;
-    // fp32 arrays: lam, delta, v (2 slots each), scan scratch, sums of squares [2][R][2][128],
+    // fp32 arrays: lam, delta, v (2 slots each), scan scratch, sums of squares [3][R][2][128],
     // conv taps and biases of the staged channels, norm weights
     static constexpr uint32_t F_LAM = 0, F_DL = 256, F_V = 512, F_SCAN = 768, F_RED = 784,
-                              F_CW = F_RED + 2 * R * 2 * 128, F_CB = F_CW + SROW * 4, F_NW = F_CB + SROW,
+                              F_CW = F_RED + 3 * R * 2 * 128, F_CB = F_CW + SROW * 4, F_NW = F_CB + SROW,
                               F_END = F_NW + kP;
     static constexpr uint32_t OFF_BAR = OFF_MISC + ((F_END * 4 + 15) / 16) * 16;
-    static constexpr int NBAR = 12;  // bar0 bar1 barX barP barC barE2[2] barF2[2] barN2[2] (+1 slot)
+    static constexpr int NBAR = 14;  // bar0 bar1 barX barP barC barE2[2] barF2[2] barN3[3] barTB barTX
     static constexpr uint32_t OFF_TSLOT = OFF_BAR + NBAR * 8;
     static constexpr uint32_t TOTAL = OFF_TSLOT + 16;
 };
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
-// Arrive on the mbarrier at `mbar_cluster` (a shared::cluster address, possibly a peer's)
-// without ordering this thread's earlier memory operations: used to say that this CTA's
-// MMAs, already seen complete, no longer read its B'/C' tiles.
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t mbar_cluster)
-{
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar_cluster) : "memory");
-}
 
 // 4-byte store into a peer's shared memory that completes 4 transaction bytes on the
 // peer's mbarrier (both shared::cluster addresses).
@@ -117,10 +118,24 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t mbar, uint32_t parity
     }
 }
 
-// Inclusive scan over threads 0..127 (warps 0..3; named barrier kBarScan).
+// Non-blocking test of a barrier phase, acquiring at cluster scope when it has completed.
+__device__ __forceinline__ bool mbar_test_cluster(uint32_t mbar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Inclusive scan over the 128 threads of warps 4..7 (named barrier kBarScan).
 __device__ __forceinline__ float scan128(float v, float* tot)
 {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, wid = (threadIdx.x >> 5) - 4;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float n = __shfl_up_sync(0xffffffffu, v, o);
@@ -133,8 +148,13 @@ __device__ __forceinline__ float scan128(float v, float* tot)
     return v + off;
 }
 
+// Tensor maps of x, B and C as [b][L][channels] (bf16), boxes of 8 channels x 128 tokens.
+struct WsMaps {
+    CUtensorMap x, B, C;
+};
+
 template <int R, bool SPLIT>
-__global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillParams p)
+__global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillParams p, const __grid_constant__ WsMaps maps)
 {
     using Lo = WsLayout<R>;
     constexpr int NS = Lo::NS, SROW = Lo::SROW;
@@ -156,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     float* s_dl = mf + Lo::F_DL;
     float* s_v = mf + Lo::F_V;
     float* s_scan = mf + Lo::F_SCAN;
-    float* s_red = mf + Lo::F_RED;     // [2 slots][R CTAs][2 halves][128 rows]
+    float* s_red = mf + Lo::F_RED;     // [3 slots][R CTAs][2 halves][128 rows]
     float* s_cw = mf + Lo::F_CW;
     float* s_cb = mf + Lo::F_CB;
     float* s_nw = mf + Lo::F_NW;
@@ -169,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const uint32_t aX = s_base + Lo::OFF_X, aXW = s_base + Lo::OFF_XW, aH = s_base + Lo::OFF_H;
     const uint32_t bar0 = smem_u32(&bars[0]), bar1 = smem_u32(&bars[1]), barX = smem_u32(&bars[2]);
     const uint32_t barP = smem_u32(&bars[3]), barC = smem_u32(&bars[4]);
-    const uint32_t barE2 = smem_u32(&bars[5]), barF2 = smem_u32(&bars[7]), barN2 = smem_u32(&bars[9]);
+    const uint32_t barE2 = smem_u32(&bars[5]), barF2 = smem_u32(&bars[7]), barN3 = smem_u32(&bars[9]);
+    const uint32_t barTB = smem_u32(&bars[12]), barTX = smem_u32(&bars[13]);   // raw B/C rows, raw x rows
 
     auto staged_channel = [&](int c) -> int64_t {
         if (c < kP) return (int64_t)h * kP + c;
@@ -191,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         const int k = e / SROW, c = e % SROW;
         __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
         if (p.init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(bi * Cc + staged_channel(c)) * 3 + k];
-        reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + k)[c % 8] = v;
+        reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + k)[c % 8] = v;
     }
     if (tid == 0) {
         mbar_init(bar0, 1);
@@ -203,9 +224,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         mbar_init(barE2 + 8, 1);
         mbar_init(barF2, R);
         mbar_init(barF2 + 8, R);
-        mbar_init(barN2, 1);
-        mbar_init(barN2 + 8, 1);
+        mbar_init(barN3, 1);
+        mbar_init(barN3 + 8, 1);
+        mbar_init(barN3 + 16, 1);
+        mbar_init(barTB, 1);
+        mbar_init(barTX, 1);
         fence_mbar_init();
+        prefetch_tmap(&maps.x);
+        prefetch_tmap(&maps.B);
+        prefetch_tmap(&maps.C);
     }
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
 
@@ -250,137 +277,180 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
 
     if (!consumer) {
         // =========================== producer (warps 0..7) ===========================
-        auto load_block = [&](int64_t k, int t0i, int nthr) {
-            const int64_t t0 = k * kT;
-            const int len = blen(k);
-            constexpr int CPR = SROW / 8;
-            for (int e = t0i; e < len * CPR; e += nthr) {
-                const int r = e / CPR, c8 = (e % CPR) * 8;
-                const int64_t tok = bi * p.L + t0 + r;
-                const __nv_bfloat16* src;
-                if (c8 < kP) src = gx + tok * p.x_ld + (int64_t)h * kP + c8;
-                else if (c8 < kP + NS) src = gB + tok * p.B_ld + (int64_t)g * kN + (int64_t)q * NS + (c8 - kP);
-                else src = gC + tok * p.C_ld + (int64_t)g * kN + (int64_t)q * NS + (c8 - kP - NS);
-                cp_async16(smem_u32(stage + (c8 / 8) * kStageRows + r + 3), src);
+        constexpr int kVX = kP / 8, kVBC = 2 * NS / 8;   // x vectors, then this CTA's B and C vectors
+        // raw rows of block kb (TMA, one box per staged vector): this CTA's B/C vectors on barTB,
+        // the head's x vectors on barTX; rows past the sequence's end read as zeros
+        auto load_bc = [&](int64_t kb) {
+            fence_async_smem();
+            mbar_arrive_expect_tx(barTB, (uint32_t)kVBC * kT * 16);
+            const int t0 = (int)(kb * kT);
+#pragma unroll 1
+            for (int v = 0; v < kVBC; ++v) {
+                const int n = q * NS + (v % (NS / 8)) * 8;
+                tma_load_3d(smem_u32(stage + (kVX + v) * kStageRows + kStageTok), v < NS / 8 ? (const void*)&maps.B : (const void*)&maps.C,
+                            g * kN + n, t0, (int)bi, barTB);
             }
-            cp_async_commit();
         };
+        auto load_x = [&](int64_t kb) {
+            fence_async_smem();
+            mbar_arrive_expect_tx(barTX, (uint32_t)kVX * kT * 16);
+            const int t0 = (int)(kb * kT);
+#pragma unroll 1
+            for (int v = 0; v < kVX; ++v)
+                tma_load_3d(smem_u32(stage + v * kStageRows + kStageTok), &maps.x, h * kP + v * 8, t0, (int)bi, barTX);
+        };
+        // softplus and cumsum of block kb into its slot (warps 4..7, token tid - 128), then dt of
+        // block kb + 1, a whole block ahead of its use
         float dt_next = 0.0f;
+        const int tok = tid - 128;
+        auto scan_block = [&](int64_t kb) {
+            const int slb = (int)(kb & 1);
+            float dl = 0.0f, a2 = 0.0f;
+            if (tok < blen(kb)) {
+                dl = softplus(dt_next + bias);
+                a2 = dl * A2;
+            }
+            if (kb + 1 < nblk && (kb + 1) * kT + tok < p.L)
+                dt_next = __bfloat162float(gdt[(bi * p.L + (kb + 1) * kT + tok) * p.dt_ld + h]);
+            const float lam = scan128(a2, s_scan);
+            s_lam[slb * kT + tok] = lam;
+            s_dl[slb * kT + tok] = dl;
+            // exp2(lam_i - lam_j) = exp2(lam_i) * exp2(-lam_j) while every factor stays a
+            // normal fp32 number (rows with lam_i > -96); chosen per row from its past only
+            s_v[slb * kT + tok] = (lam > -96.0f) ? ex2(-lam) * dl : 0.0f;
+        };
         if (nblk > 0) {
-            load_block(0, tid, kProd);
-            if (tid < kT && tid < p.L) dt_next = __bfloat162float(gdt[(bi * p.L + tid) * p.dt_ld + h]);
+            if (tid == 0) {
+                load_bc(0);
+                load_x(0);
+            }
+            if (warp >= 4) {
+                if (tok < p.L) dt_next = __bfloat162float(gdt[(bi * p.L + tok) * p.dt_ld + h]);
+                scan_block(0);
+            }
         }
         for (int64_t k = 0; k < nblk; ++k) {
             const int len = blen(k);
             const int sl = (int)(k & 1);
-            // buffers of this block: x'[sl] and the cumsum slot were last read by the
-            // consumer in block k-2; B'/C'/x'w by this CTA's MMAs of block k-1
+            // buffers of this block: x'[sl] was last read by the consumer in block k-2, B'/C'/x'w
+            // by this CTA's MMAs of block k-1; the cumsum of this block is already in its slot
             if (tid == 0) {
                 if (k >= 1 && ok && !mbar_wait_bounded(bar0, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
                 if (k >= 2 && ok && !mbar_wait_bounded(barE2 + 8 * sl, (uint32_t)(((k - 2) >> 1) & 1), kWaitLimit)) ok = false;
+                mbar_arrive_expect_tx(barX, (uint32_t)(R - 1) * 2 * kSliceBytes);
             }
-            cp_async_wait_all();
-            named_sync(kBarProd, kProd);
-            // softplus and cumsum of this block (warps 0..3)
-            if (tid < kT) {
-                float dl = 0.0f, a2 = 0.0f;
-                if (tid < len) {
-                    dl = softplus(dt_next + bias);
-                    a2 = dl * A2;
-                }
-                const float lam = scan128(a2, s_scan);
-                s_lam[sl * kT + tid] = lam;
-                s_dl[sl * kT + tid] = dl;
-                // exp2(lam_i - lam_j) = exp2(lam_i) * exp2(-lam_j) while every factor stays a
-                // normal fp32 number (rows with lam_i > -96); chosen per row from its past only
-                s_v[sl * kT + tid] = (lam > -96.0f) ? ex2(-lam) * dl : 0.0f;
-            }
-            if (tid == 0) mbar_arrive_expect_tx(barX, (uint32_t)(R - 1) * 2 * kSliceBytes);
+            // this block's raw B/C rows (its x rows may still be in flight)
+            if (ok && !mbar_wait_bounded(barTB, (uint32_t)(k & 1), kWaitLimit)) ok = false;
             named_sync(kBarProd, kProd);
             const float* lamb = s_lam + sl * kT;
             const float* dlb = s_dl + sl * kT;
             const float lam_end = lamb[kT - 1];
-            // conv + SiLU: x' and x'w of this head, this CTA's slice of B' and C'
-            {
+            // conv + SiLU of the staged 8-channel vectors [vbeg, vbeg + VC): x' and x'w of this
+            // head, or this CTA's slice of B' and C'. TPV threads per vector, each taking rows
+            // i = t % TPV + TPV m, so a warp reads consecutive staged rows and writes
+            // consecutive canonical rows (conflict-free); a thread keeps its taps in registers.
+            auto conv_vectors = [&](auto vbeg_c, auto vc_c) {
+                constexpr int VBEG = decltype(vbeg_c)::value, VC = decltype(vc_c)::value;
+                constexpr int TPV = kProd / VC;
+                static_assert(kProd % VC == 0 && kT % (2 * TPV) == 0, "conv work split");
                 unsigned char* sX = smem + Lo::OFF_X + sl * 16384;
                 unsigned char* sXW = smem + Lo::OFF_XW;
-                // Work split: 16 threads per 8-channel vector v, each taking rows i = t%16 + 16m,
-                // so a warp covers 16 consecutive rows of 2 vectors (conflict-free staged reads
-                // and canonical stores) and a thread keeps its vector's taps in registers.
-                constexpr int kPasses = (Lo::NV + 15) / 16;
-                for (int pass = 0; pass < kPasses; ++pass) {
-                    const int v = pass * 16 + tid / 16;
-                    if (v >= Lo::NV) break;
-                    const int c0 = v * 8;
-                    float2 wr[4][4], br[4];
-                    {
-                        const float2* cw2 = reinterpret_cast<const float2*>(s_cw) + (c0 / 2) * 4;
-                        const float2* cb2 = reinterpret_cast<const float2*>(s_cb) + c0 / 2;
+                const int v = VBEG + tid / TPV;
+                const int c0 = v * 8;
+                float2 wr[4][4], br[4];
+                {
+                    const float2* cw2 = reinterpret_cast<const float2*>(s_cw) + (c0 / 2) * 4;
+                    const float2* cb2 = reinterpret_cast<const float2*>(s_cb) + c0 / 2;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            br[j] = cb2[j];
+                    for (int j = 0; j < 4; ++j) {
+                        br[j] = cb2[j];
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) wr[j][kk] = cw2[j * 4 + kk];
-                        }
+                        for (int kk = 0; kk < 4; ++kk) wr[j][kk] = cw2[j * 4 + kk];
                     }
-                    const bool is_x = c0 < kP;
-                    const bool isC = c0 >= kP + NS;
-                    const int n0 = q * NS + (isC ? c0 - kP - NS : c0 - kP);
-                    unsigned char* dstBC = smem + (isC ? Lo::OFF_C : Lo::OFF_B);
+                }
+                const bool is_x = c0 < kP;
+                const bool isC = c0 >= kP + NS;
+                const int n0 = q * NS + (isC ? c0 - kP - NS : c0 - kP);
+                unsigned char* dstBC = smem + (isC ? Lo::OFF_C : Lo::OFF_B);
 #pragma unroll 1
-                    for (int m = 0; m < 8; m += 2) {
-                        int ii[2];
-                        uint4 raw[2][4];
+                for (int m = 0; m < kT / TPV; m += 2) {
+                    int ii[2];
+                    uint4 raw[2][4];
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            ii[u] = (tid % 16) + 16 * (m + u);
+                    for (int u = 0; u < 2; ++u) {
+                        ii[u] = (tid % TPV) + TPV * (m + u);
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) raw[u][kk] = stage[v * kStageRows + ii[u] + kk];
+                        for (int kk = 0; kk < 4; ++kk) raw[u][kk] = stage[v * kStageRows + kStageTok - 3 + ii[u] + kk];
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int i = ii[u];
+                        float2 o[4];
+                        if (i < len) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {   // channel pair (c0 + 2j, c0 + 2j + 1)
+                                float2 vv = fma2(wr[j][0], bf2_to_f2((&raw[u][0].x)[j]), br[j]);
+                                vv = fma2(wr[j][1], bf2_to_f2((&raw[u][1].x)[j]), vv);
+                                vv = fma2(wr[j][2], bf2_to_f2((&raw[u][2].x)[j]), vv);
+                                vv = fma2(wr[j][3], bf2_to_f2((&raw[u][3].x)[j]), vv);
+                                o[j] = silu2(vv);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) o[j] = make_float2(0.0f, 0.0f);
                         }
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int i = ii[u];
-                            float2 o[4];
-                            if (i < len) {
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {   // channel pair (c0 + 2j, c0 + 2j + 1)
-                                    float2 vv = fma2(wr[j][0], bf2_to_f2((&raw[u][0].x)[j]), br[j]);
-                                    vv = fma2(wr[j][1], bf2_to_f2((&raw[u][1].x)[j]), vv);
-                                    vv = fma2(wr[j][2], bf2_to_f2((&raw[u][2].x)[j]), vv);
-                                    vv = fma2(wr[j][3], bf2_to_f2((&raw[u][3].x)[j]), vv);
-                                    o[j] = silu2(vv);
-                                }
-                            } else {
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) o[j] = make_float2(0.0f, 0.0f);
-                            }
-                            const uint4 u8 = make_uint4(pack_f2(o[0]), pack_f2(o[1]), pack_f2(o[2]), pack_f2(o[3]));
-                            if (is_x) {
-                                const float2 wgt = splat2((i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f);
-                                const uint4 uw = make_uint4(pack_f2(mul2(o[0], wgt)), pack_f2(mul2(o[1], wgt)),
-                                                            pack_f2(mul2(o[2], wgt)), pack_f2(mul2(o[3], wgt)));
-                                *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
-                                *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
-                            } else {
-                                *reinterpret_cast<uint4*>(dstBC + canon_koff(i, n0, kT)) = u8;
-                            }
+                        const uint4 u8 = make_uint4(pack_f2(o[0]), pack_f2(o[1]), pack_f2(o[2]), pack_f2(o[3]));
+                        if (is_x) {
+                            const float2 wgt = splat2((i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f);
+                            const uint4 uw = make_uint4(pack_f2(mul2(o[0], wgt)), pack_f2(mul2(o[1], wgt)),
+                                                        pack_f2(mul2(o[2], wgt)), pack_f2(mul2(o[3], wgt)));
+                            *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
+                            *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
+                        } else {
+                            *reinterpret_cast<uint4*>(dstBC + canon_koff(i, n0, kT)) = u8;
                         }
                     }
                 }
-            }
+            };
+            // this CTA's slice of B' and C' first, so its copies to the peers overlap the x' conv
+            conv_vectors(std::integral_constant<int, kVX>{}, std::integral_constant<int, kVBC>{});
             fence_async_smem();
             named_sync(kBarProd, kProd);
-            if (tid == 0) {
-                // the peers' MMAs of block k-1 are done: their B'/C' may take this block's slice
-                if (k >= 1 && ok &&
-                    !mbar_wait_cluster(barF2 + 8 * ((k - 1) & 1), (uint32_t)(((k - 1) >> 1) & 1), kWaitLimit))
-                    ok = false;
+            // the B/C raw rows of this block are consumed: their halo, then the next block's rows
+            if (k + 1 < nblk) {
+                for (int e = tid; e < 3 * kVBC; e += kProd) {
+                    const int r = e % 3, v = kVX + e / 3;
+                    stage[v * kStageRows + kStageTok - 3 + r] = stage[v * kStageRows + kStageTok + kT - 3 + r];
+                }
+                named_sync(kBarHalo, kProd);
+                if (tid == 0) load_bc(k + 1);
+            }
+            // this CTA's slice of B'/C' to every peer, once the peers' MMAs of block k-1 no longer
+            // read their B'/C': now if that is already so, else after the x' conv
+            auto send_slice = [&]() {
 #pragma unroll
                 for (int rr = 0; rr < R; ++rr) {
                     if (rr == q) continue;
                     const uint32_t mb = cluster_map(barX, (uint32_t)rr);
                     bulk_copy_to_peer(cluster_map(aB + slice_off, (uint32_t)rr), aB + slice_off, kSliceBytes, mb);
                     bulk_copy_to_peer(cluster_map(aC + slice_off, (uint32_t)rr), aC + slice_off, kSliceBytes, mb);
+                }
+            };
+            const uint32_t barF_prev = barF2 + 8 * (uint32_t)((k - 1) & 1), parF_prev = (uint32_t)(((k - 1) >> 1) & 1);
+            bool sent = false;
+            if (tid == 0 && (k == 0 || mbar_test_cluster(barF_prev, parF_prev))) {
+                send_slice();
+                sent = true;
+            }
+            // this block's raw x rows (the next block's B/C rows may be in flight)
+            if (ok && !mbar_wait_bounded(barTX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
+            conv_vectors(std::integral_constant<int, 0>{}, std::integral_constant<int, kVX>{});
+            fence_async_smem();
+            named_sync(kBarProd, kProd);
+            if (tid == 0) {
+                if (!sent) {
+                    if (ok && !mbar_wait_cluster(barF_prev, parF_prev, kWaitLimit)) ok = false;
+                    send_slice();
                 }
                 if (ok && !mbar_wait_bounded(barX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
                 // the consumer has read C'B'^T and S^T of block k-1 and written H^T for this block
@@ -401,18 +471,27 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16(tmem + kColS, sdesc(aB + kk * 256, 128, 2048), sdesc(aXW + kk * 2048, 1024, 128), id_s, kk > 0);
                 mma_commit(bar0);
+                // once these MMAs are done, this CTA's B'/C' may be overwritten: every peer is told
+                mma_commit_cluster(barF2 + 8 * (uint32_t)sl, (uint16_t)((1u << R) - 1));
             }
-            // raw rows of the next block (warps 1..7): halo, then the loads; dt of the next block
-            if (k + 1 < nblk && warp > 0) {
-                for (int e = tid - 32; e < 3 * Lo::NV; e += kProd - 32) {
-                    const int r = e % 3, v = e / 3;
-                    stage[v * kStageRows + r] = stage[v * kStageRows + kT + r];
+            // while thread 0 issues the MMAs: x raw rows of the next block (warps 1..3) and its
+            // softplus and cumsum (warps 4..7, once the consumer has released that slot in block k-1)
+            if (k + 1 < nblk) {
+                if (warp >= 1 && warp < 4) {
+                    for (int e = tid - 32; e < 3 * kVX; e += 96) {
+                        const int r = e % 3, v = e / 3;
+                        stage[v * kStageRows + kStageTok - 3 + r] = stage[v * kStageRows + kStageTok + kT - 3 + r];
+                    }
+                    named_sync(kBarHaloX, 96);
+                    if (tid == 32) load_x(k + 1);
+                } else if (warp >= 4) {
+                    if (k >= 1 && tid == 128 && ok &&
+                        !mbar_wait_bounded(barE2 + 8 * ((k + 1) & 1), (uint32_t)(((k - 1) >> 1) & 1), kWaitLimit))
+                        ok = false;
+                    named_sync(kBarScan, 128);
+                    scan_block(k + 1);
                 }
-                named_sync(kBarHalo, kProd - 32);
-                load_block(k + 1, tid - 32, kProd - 32);
             }
-            if (k + 1 < nblk && tid < kT && (k + 1) * kT + tid < p.L)
-                dt_next = __bfloat162float(gdt[(bi * p.L + (k + 1) * kT + tid) * p.dt_ld + h]);
         }
         // final conv state: the last three raw inputs of the staged channels
         const int len_last = nblk > 0 ? blen(nblk - 1) : 0;
@@ -420,11 +499,40 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         for (int e = tid; e < 3 * SROW; e += kProd) {
             const int kk = e / SROW, c = e % SROW;
             ((__nv_bfloat16*)p.final_conv)[(bi * Cc + staged_channel(c)) * 3 + kk] =
-                reinterpret_cast<const __nv_bfloat16*>(stage + (c / 8) * kStageRows + len_last + kk)[c % 8];
+                reinterpret_cast<const __nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + len_last + kk)[c % 8];
         }
     } else {
         // =========================== consumer (warps 8..15) ===========================
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        // 32 output channels of one row: gated values, optionally scaled by the norm and weighted
+        auto store_y = [&](__nv_bfloat16* dst, const float* gv, float scale, bool norm) {
+            uint4* yo = reinterpret_cast<uint4*>(dst);
+            const float2* nw2 = reinterpret_cast<const float2*>(s_nw + chalf * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 gg = make_float2(gv[8 * v + 2 * e], gv[8 * v + 2 * e + 1]);
+                    w[e] = pack_f2(norm ? mul2(mul2(gg, splat2(scale)), nw2[4 * v + e]) : gg);
+                }
+                yo[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        };
+        // group RMSNorm of block kb: every CTA's sums of squares, the gated values from TMEM
+        auto finish_norm = [&](int64_t kb) {
+            const uint32_t nsl = (uint32_t)(kb % 3);
+            if (ok && !mbar_wait_cluster(barN3 + 8 * nsl, (uint32_t)((kb / 3) & 1), kWaitLimit)) ok = false;
+            float tot = 0.0f;
+#pragma unroll
+            for (int rr = 0; rr < 2 * R; ++rr) tot += s_red[(nsl * R * 2 + rr) * 128 + crow];
+            const float scale = rsqrtf(tot / (float)(R * kP) + p.eps);
+            float gv[32];
+            tmem_ld32(tmem + lane_base + kColG + chalf * 32, gv);
+            tmem_wait_ld();
+            if (crow < blen(kb))
+                store_y(gy + (bi * p.L + kb * kT + crow) * p.y_ld + (int64_t)h * kP + chalf * 32, gv, scale, true);
+        };
         for (int64_t k = 0; k < nblk; ++k) {
             const int64_t t0 = k * kT;
             const int len = blen(k);
@@ -443,12 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             if (ok && !mbar_wait_bounded(barP, par, kWaitLimit)) ok = false;
             if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
             fence_after_sync();
-            // this CTA's MMAs on B'/C' of block k are done: tell every peer; and expect the
-            // peers' sums of squares of block k (2 floats per row from every CTA)
-            if (tid == kProd) {
-#pragma unroll
-                for (int rr = 0; rr < R; ++rr) mbar_arrive_remote_relaxed(cluster_map(barF2 + 8 * sl, (uint32_t)rr));
-                if constexpr (!SPLIT) mbar_arrive_expect_tx(barN2 + 8 * sl, (uint32_t)(R * 2 * 128 * 4));
+            // expect the peers' sums of squares of block k (2 floats per row from every CTA)
+            if constexpr (!SPLIT) {
+                if (tid == kProd) mbar_arrive_expect_tx(barN3 + 8 * (uint32_t)(k % 3), (uint32_t)(R * 2 * 128 * 4));
             }
             const float* lamb = s_lam + sl * kT;
             const float* dlb = s_dl + sl * kT;
@@ -532,6 +637,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     mma_bf16(tmem + kColYi, sdesc(aM + kk * 256, 128, 2048), sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
                 mma_commit(bar1);
             }
+            if constexpr (!SPLIT) {
+                if (k >= 1) finish_norm(k - 1);   // overlaps the MMA M x' of this block
+            }
             if (ok && !mbar_wait_bounded(bar1, par, kWaitLimit)) ok = false;
             fence_after_sync();
             // epilogue: y = Yi + exp(lam_i) Ys + D x', gate
@@ -563,37 +671,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 if constexpr (SPLIT) {
                     if (i < len) p.ssp[((bi * p.L + t0 + i) * p.H + h) * 2 + chalf] = ss;
                 } else {
-                    const uint32_t dst = smem_u32(s_red + ((sl * R + q) * 2 + chalf) * 128 + i);
+                    const uint32_t nsl = (uint32_t)(k % 3);
+                    const uint32_t dst = smem_u32(s_red + ((nsl * R + q) * 2 + chalf) * 128 + i);
 #pragma unroll
                     for (int rr = 0; rr < R; ++rr)
-                        st_async_f32(cluster_map(dst, (uint32_t)rr), ss, cluster_map(barN2 + 8 * sl, (uint32_t)rr));
+                        st_async_f32(cluster_map(dst, (uint32_t)rr), ss, cluster_map(barN3 + 8 * nsl, (uint32_t)rr));
+                    tmem_st32(tmem + lane_base + kColG + chalf * 32, gt);
+                    tmem_wait_st();
                 }
             }
             fence_before_sync();
             named_sync(kBarCons, kThreads - kProd);
             if (tid == kProd) mbar_arrive_local(barE2 + 8 * sl);   // x'[sl] and the cumsum slot are free
-            float scale = 1.0f;
-            if constexpr (!SPLIT) {
-                if (ok && !mbar_wait_cluster(barN2 + 8 * sl, (uint32_t)((k >> 1) & 1), kWaitLimit)) ok = false;
-                float tot = 0.0f;
-#pragma unroll
-                for (int rr = 0; rr < 2 * R; ++rr) tot += s_red[(sl * R * 2 + rr) * 128 + crow];
-                scale = rsqrtf(tot / (float)(R * kP) + p.eps);
+            if constexpr (SPLIT) {
+                if (crow < len) store_y(gy + (bi * p.L + t0 + crow) * p.y_ld + (int64_t)h * kP + chalf * 32, gt, 1.0f, false);
             }
-            if (crow < len) {
-                uint4* yo = reinterpret_cast<uint4*>(gy + (bi * p.L + t0 + crow) * p.y_ld + (int64_t)h * kP + chalf * 32);
-                const float2* nw2 = reinterpret_cast<const float2*>(s_nw + chalf * 32);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 gg = make_float2(gt[8 * v + 2 * e], gt[8 * v + 2 * e + 1]);
-                        w[e] = pack_f2(SPLIT ? gg : mul2(mul2(gg, splat2(scale)), nw2[4 * v + e]));
-                    }
-                    yo[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
+        }
+        if constexpr (!SPLIT) {
+            if (nblk >= 1) finish_norm(nblk - 1);
         }
         // final SSM state of this head
         float* fs = p.final_ssm + (bi * p.H + h) * (int64_t)kP * kN;
@@ -636,10 +731,49 @@ __global__ void __launch_bounds__(256) ws_norm_finish_kernel(PrefillParams p)
     }
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime (no link-time libcuda dependency).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn()
+{
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+// [b][L][width] bf16 rows of `ld` elements; boxes of 8 channels x 128 tokens x 1 sequence.
+bool encode_rows(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b)
+{
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)L, (cuuint64_t)b};
+    const cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(L * ld * 2)};
+    const cuuint32_t box[3] = {8, (cuuint32_t)kT, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int R, bool SPLIT>
 cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
 {
     using Lo = WsLayout<R>;
+    WsMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (p.L > 0) {   // no block, no load: the maps stay unused
+        if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, p.L, p.b) || !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, p.L, p.b) ||
+            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, p.L, p.b))
+            return cudaErrorInvalidValue;
+    }
     cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::TOTAL);
     if (e != cudaSuccess) return e;
@@ -657,7 +791,7 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     cfg.numAttrs = 1;
     {
         LaunchScope ls("tc_prefill", st);
-        e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT>, p);
+        e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT>, p, maps);
         if (e != cudaSuccess) return e;
     }
     if (SPLIT && p.L > 0) {

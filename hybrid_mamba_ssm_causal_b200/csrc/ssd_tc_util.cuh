@@ -1,5 +1,5 @@
 // ssd_tc_util.cuh -- sm_100a building blocks: tcgen05 MMA with TMEM accumulators, shared
-// memory matrix descriptors, mbarriers with bounded waits, TMEM loads, cp.async.
+// memory matrix descriptors, mbarriers with bounded waits, TMEM loads, TMA and cp.async.
 //
 // Operand tiles live in shared memory in the no-swizzle canonical layout: 8x8 bf16 "core
 // matrices" of 128 contiguous bytes (8 rows of 16 bytes), stored block-row-major with the
@@ -44,6 +44,21 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank)
 
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into a peer CTA's
 // shared memory; completes `bytes` of transaction count on the peer's mbarrier.
+// Tiled bulk-tensor load (TMA) of one box of a 3-D tensor map into this CTA's shared memory,
+// completing its bytes on `mbar`. The box's innermost extent times the element size is a
+// multiple of 16 bytes and c0 (innermost coordinate) times the element size too.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2, uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const void* tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
                                                   uint32_t mbar_cluster)
 {
@@ -96,6 +111,15 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
 __device__ __forceinline__ void mma_commit(uint32_t mbar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+// Arrive once on the mbarrier at the same shared-memory offset in every CTA of `cta_mask`
+// when all previously issued tcgen05 operations of this thread have completed.
+__device__ __forceinline__ void mma_commit_cluster(uint32_t mbar, uint16_t cta_mask)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(mbar), "h"(cta_mask)
                  : "memory");
 }
 
@@ -199,6 +223,27 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v)
     else tmem_ld32(taddr, v);
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Store 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 16-byte global -> shared asynchronous copy (L2 only) and its group fences.
 __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src)
@@ -207,6 +252,8 @@ __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src)
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// All but the most recent committed group of this thread have landed.
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // sigmoid(v) * v with the hardware tanh approximation (relative error ~2^-11, below
 // the bf16 rounding of the result).
