@@ -57,8 +57,9 @@ constexpr int kP = 64;        // head dim
 constexpr int kN = 128;       // state dim
 constexpr int kThreads = 512;
 constexpr int kProd = 256;    // producer threads (warps 0..7)
-// Raw staging of one 8-channel vector: rows 5..7 hold the three tokens before the block
-// (the conv halo), rows 8..135 the block's tokens (one TMA box, 128-byte aligned).
+// Raw staging of one 8-channel vector: tokens t0-8 .. t0+127 of a block, so rows 5..7 hold
+// the conv halo and rows 8..135 the block's tokens; 2176 bytes, a multiple of 128, so every
+// vector starts 128-byte aligned. One TMA box fills several consecutive vectors.
 constexpr int kStageRows = 136, kStageTok = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
@@ -67,7 +68,7 @@ constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
 constexpr uint32_t kColCB = 0, kColYs0 = 128, kColS = 256, kColYi = 320, kColG = 384;
 
 // named barriers
-constexpr int kBarProd = 1, kBarCons = 2, kBarScan = 3, kBarHalo = 4, kBarHaloX = 5;
+constexpr int kBarProd = 1, kBarCons = 2, kBarScan = 3;
 
 template <int R>
 struct WsLayout {
@@ -148,7 +149,8 @@ __device__ __forceinline__ float scan128(float v, float* tot)
     return v + off;
 }
 
-// Tensor maps of x, B and C as [b][L][channels] (bf16), boxes of 8 channels x 128 tokens.
+// Tensor maps of x, B and C viewed as [b][vector][token][8 channels] (bf16; a vector is 8
+// consecutive channels), boxes of 136 tokens x several vectors.
 struct WsMaps {
     CUtensorMap x, B, C;
 };
@@ -208,12 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         s_cb[c] = p.conv_b[ch];
     }
     if (tid < kP) s_nw[tid] = p.norm_w[(int64_t)h * kP + tid];
-    for (int e = tid; e < 3 * SROW; e += kThreads) {
-        const int k = e / SROW, c = e % SROW;
-        __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
-        if (p.init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(bi * Cc + staged_channel(c)) * 3 + k];
-        reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + k)[c % 8] = v;
-    }
     if (tid == 0) {
         mbar_init(bar0, 1);
         mbar_init(bar1, 1);
@@ -278,26 +274,17 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     if (!consumer) {
         // =========================== producer (warps 0..7) ===========================
         constexpr int kVX = kP / 8, kVBC = 2 * NS / 8;   // x vectors, then this CTA's B and C vectors
-        // raw rows of block kb (TMA, one box per staged vector): this CTA's B/C vectors on barTB,
-        // the head's x vectors on barTX; rows past the sequence's end read as zeros
+        // raw rows t0-8 .. t0+127 of block kb (TMA): one box for the head's x vectors on barTX, one
+        // each for this CTA's B and C vectors on barTB; rows outside the sequence read as zeros
         auto load_bc = [&](int64_t kb) {
-            fence_async_smem();
-            mbar_arrive_expect_tx(barTB, (uint32_t)kVBC * kT * 16);
-            const int t0 = (int)(kb * kT);
-#pragma unroll 1
-            for (int v = 0; v < kVBC; ++v) {
-                const int n = q * NS + (v % (NS / 8)) * 8;
-                tma_load_3d(smem_u32(stage + (kVX + v) * kStageRows + kStageTok), v < NS / 8 ? (const void*)&maps.B : (const void*)&maps.C,
-                            g * kN + n, t0, (int)bi, barTB);
-            }
+            mbar_arrive_expect_tx(barTB, (uint32_t)kVBC * kStageRows * 16);
+            const int t0 = (int)(kb * kT) - kStageTok, vb = (g * kN + q * NS) / 8;
+            tma_load_4d(smem_u32(stage + kVX * kStageRows), &maps.B, 0, t0, vb, (int)bi, barTB);
+            tma_load_4d(smem_u32(stage + (kVX + NS / 8) * kStageRows), &maps.C, 0, t0, vb, (int)bi, barTB);
         };
         auto load_x = [&](int64_t kb) {
-            fence_async_smem();
-            mbar_arrive_expect_tx(barTX, (uint32_t)kVX * kT * 16);
-            const int t0 = (int)(kb * kT);
-#pragma unroll 1
-            for (int v = 0; v < kVX; ++v)
-                tma_load_3d(smem_u32(stage + v * kStageRows + kStageTok), &maps.x, h * kP + v * 8, t0, (int)bi, barTX);
+            mbar_arrive_expect_tx(barTX, (uint32_t)kVX * kStageRows * 16);
+            tma_load_4d(smem_u32(stage), &maps.x, 0, (int)(kb * kT) - kStageTok, h * kVX, (int)bi, barTX);
         };
         // softplus and cumsum of block kb into its slot (warps 4..7, token tid - 128), then dt of
         // block kb + 1, a whole block ahead of its use
@@ -327,6 +314,20 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             if (warp >= 4) {
                 if (tok < p.L) dt_next = __bfloat162float(gdt[(bi * p.L + tok) * p.dt_ld + h]);
                 scan_block(0);
+            }
+        }
+        // the three rows before the sequence hold the initial conv state (zeros without one), not
+        // the TMA's fill: written once block 0's rows have landed
+        if (nblk == 0 || p.init_conv) {
+            if (nblk > 0) {
+                if (ok && !mbar_wait_bounded(barTB, 0, kWaitLimit)) ok = false;
+                if (ok && !mbar_wait_bounded(barTX, 0, kWaitLimit)) ok = false;
+            }
+            for (int e = tid; e < 3 * SROW; e += kProd) {
+                const int kk = e / SROW, c = e % SROW;
+                __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
+                if (p.init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(bi * Cc + staged_channel(c)) * 3 + kk];
+                reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + kk)[c % 8] = v;
             }
         }
         for (int64_t k = 0; k < nblk; ++k) {
@@ -416,42 +417,36 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             conv_vectors(std::integral_constant<int, kVX>{}, std::integral_constant<int, kVBC>{});
             fence_async_smem();
             named_sync(kBarProd, kProd);
-            // the B/C raw rows of this block are consumed: their halo, then the next block's rows
-            if (k + 1 < nblk) {
-                for (int e = tid; e < 3 * kVBC; e += kProd) {
-                    const int r = e % 3, v = kVX + e / 3;
-                    stage[v * kStageRows + kStageTok - 3 + r] = stage[v * kStageRows + kStageTok + kT - 3 + r];
-                }
-                named_sync(kBarHalo, kProd);
-                if (tid == 0) load_bc(k + 1);
-            }
-            // this CTA's slice of B'/C' to every peer, once the peers' MMAs of block k-1 no longer
-            // read their B'/C': now if that is already so, else after the x' conv
+            // this CTA's slice of B'/C' to every peer (warp 0, one copy per lane), once the peers'
+            // MMAs of block k-1 no longer read their B'/C': now if that is already so, else after
+            // the x' conv; and (lane 0) the next block's raw B/C rows, now that these are consumed
+            const int lane = tid & 31;
             auto send_slice = [&]() {
-#pragma unroll
-                for (int rr = 0; rr < R; ++rr) {
-                    if (rr == q) continue;
-                    const uint32_t mb = cluster_map(barX, (uint32_t)rr);
-                    bulk_copy_to_peer(cluster_map(aB + slice_off, (uint32_t)rr), aB + slice_off, kSliceBytes, mb);
-                    bulk_copy_to_peer(cluster_map(aC + slice_off, (uint32_t)rr), aC + slice_off, kSliceBytes, mb);
+                if (lane >= 1 && lane <= 2 * (R - 1)) {
+                    const int idx = lane - 1;
+                    const uint32_t rr = (uint32_t)((q + 1 + idx / 2) % R);
+                    const uint32_t src = (idx & 1 ? aC : aB) + slice_off;
+                    bulk_copy_to_peer(cluster_map(src, rr), src, kSliceBytes, cluster_map(barX, rr));
                 }
             };
             const uint32_t barF_prev = barF2 + 8 * (uint32_t)((k - 1) & 1), parF_prev = (uint32_t)(((k - 1) >> 1) & 1);
             bool sent = false;
-            if (tid == 0 && (k == 0 || mbar_test_cluster(barF_prev, parF_prev))) {
-                send_slice();
-                sent = true;
+            if (warp == 0) {
+                if (tid == 0 && k + 1 < nblk) load_bc(k + 1);
+                sent = __shfl_sync(0xffffffffu, (int)(k == 0 || (lane == 0 && mbar_test_cluster(barF_prev, parF_prev))), 0) != 0;
+                if (sent) send_slice();
             }
             // this block's raw x rows (the next block's B/C rows may be in flight)
             if (ok && !mbar_wait_bounded(barTX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
             conv_vectors(std::integral_constant<int, 0>{}, std::integral_constant<int, kVX>{});
             fence_async_smem();
             named_sync(kBarProd, kProd);
+            if (warp == 0 && !sent) {
+                if (tid == 0 && ok && !mbar_wait_cluster(barF_prev, parF_prev, kWaitLimit)) ok = false;
+                __syncwarp();
+                send_slice();
+            }
             if (tid == 0) {
-                if (!sent) {
-                    if (ok && !mbar_wait_cluster(barF_prev, parF_prev, kWaitLimit)) ok = false;
-                    send_slice();
-                }
                 if (ok && !mbar_wait_bounded(barX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
                 // the consumer has read C'B'^T and S^T of block k-1 and written H^T for this block
                 if (k >= 1 && ok && !mbar_wait_bounded(barC, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
@@ -474,16 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 // once these MMAs are done, this CTA's B'/C' may be overwritten: every peer is told
                 mma_commit_cluster(barF2 + 8 * (uint32_t)sl, (uint16_t)((1u << R) - 1));
             }
-            // while thread 0 issues the MMAs: x raw rows of the next block (warps 1..3) and its
+            // while thread 0 issues the MMAs: x raw rows of the next block (thread 32) and its
             // softplus and cumsum (warps 4..7, once the consumer has released that slot in block k-1)
             if (k + 1 < nblk) {
-                if (warp >= 1 && warp < 4) {
-                    for (int e = tid - 32; e < 3 * kVX; e += 96) {
-                        const int r = e % 3, v = e / 3;
-                        stage[v * kStageRows + kStageTok - 3 + r] = stage[v * kStageRows + kStageTok + kT - 3 + r];
-                    }
-                    named_sync(kBarHaloX, 96);
-                    if (tid == 32) load_x(k + 1);
+                if (tid == 32) {
+                    load_x(k + 1);
                 } else if (warp >= 4) {
                     if (k >= 1 && tid == 128 && ok &&
                         !mbar_wait_bounded(barE2 + 8 * ((k + 1) & 1), (uint32_t)(((k - 1) >> 1) & 1), kWaitLimit))
@@ -749,16 +739,17 @@ EncodeTiledFn encode_tiled_fn()
     return fn;
 }
 
-// [b][L][width] bf16 rows of `ld` elements; boxes of 8 channels x 128 tokens x 1 sequence.
-bool encode_rows(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b)
+// [b][L][width] bf16 rows of `ld` elements viewed as [b][width/8 vectors][L][8]; boxes of
+// 8 channels x kStageRows tokens x `nvec` vectors x 1 sequence land as [vector][token][8].
+bool encode_rows(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b, int nvec)
 {
     EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)L, (cuuint64_t)b};
-    const cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(L * ld * 2)};
-    const cuuint32_t box[3] = {8, (cuuint32_t)kT, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    const cuuint64_t dims[4] = {8, (cuuint64_t)L, (cuuint64_t)(width / 8), (cuuint64_t)b};
+    const cuuint64_t strides[3] = {(cuuint64_t)(ld * 2), 16, (cuuint64_t)(L * ld * 2)};
+    const cuuint32_t box[4] = {8, (cuuint32_t)kStageRows, (cuuint32_t)nvec, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -770,8 +761,9 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     WsMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (p.L > 0) {   // no block, no load: the maps stay unused
-        if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, p.L, p.b) || !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, p.L, p.b) ||
-            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, p.L, p.b))
+        if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, p.L, p.b, kP / 8) ||
+            !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, p.L, p.b, Lo::NS / 8) ||
+            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, p.L, p.b, Lo::NS / 8))
             return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
