@@ -64,8 +64,9 @@ constexpr int kStageRows = 136, kStageTok = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
 
-// TMEM columns: C'B'^T, Ys (two slots), S^T, Yi, the gated values of a block awaiting its norm
-constexpr uint32_t kColCB = 0, kColYs0 = 128, kColS = 256, kColYi = 320, kColG = 384;
+// TMEM columns: C'B'^T, Ys (two slots), S^T, Yi, the gated values of a block awaiting its norm,
+// and the masked decay matrix M (bf16 pairs; the A operand of M x')
+constexpr uint32_t kColCB = 0, kColYs0 = 128, kColS = 256, kColYi = 320, kColG = 384, kColM = 448;
 
 // named barriers
 constexpr int kBarProd = 1, kBarCons = 2, kBarScan = 3;
@@ -74,8 +75,8 @@ template <int R>
 struct WsLayout {
     static constexpr int NS = kN / R;                // B/C channels convolved by one CTA
     static constexpr int SROW = kP + 2 * NS;
-    static constexpr int NV = SROW / 8;
-    static constexpr uint32_t OFF_C = 0, OFF_B = 32768, OFF_M = 65536, OFF_X = 98304,   // x' [2]
+    // z and y tiles of a block: [128 tokens][64 channels] bf16, 16-byte chunks swizzled by token % 8
+    static constexpr uint32_t OFF_C = 0, OFF_B = 32768, OFF_Z = 65536, OFF_Y = 81920, OFF_X = 98304,   // x' [2]
                               OFF_XW = OFF_X + 2 * 16384, OFF_H = OFF_XW + 16384, OFF_STAGE = OFF_H + 16384;
     static constexpr uint32_t STAGE_BYTES = (uint32_t)kStageRows * SROW * 2;   // SROW/8 vectors
     static constexpr uint32_t OFF_MISC = OFF_STAGE + ((STAGE_BYTES + 127) / 128) * 128;
@@ -85,7 +86,7 @@ struct WsLayout {
                               F_CW = F_RED + 3 * R * 2 * 128, F_CB = F_CW + SROW * 4, F_NW = F_CB + SROW,
                               F_END = F_NW + kP;
     static constexpr uint32_t OFF_BAR = OFF_MISC + ((F_END * 4 + 15) / 16) * 16;
-    static constexpr int NBAR = 14;  // bar0 bar1 barX barP barC barE2[2] barF2[2] barN3[3] barTB barTX
+    static constexpr int NBAR = 15;  // bar0 bar1 barX barP barC barE2[2] barF2[2] barN3[3] barTB barTX barZ
     static constexpr uint32_t OFF_TSLOT = OFF_BAR + NBAR * 8;
     static constexpr uint32_t TOTAL = OFF_TSLOT + 16;
 };
@@ -150,9 +151,10 @@ __device__ __forceinline__ float scan128(float v, float* tot)
 }
 
 // Tensor maps of x, B and C viewed as [b][vector][token][8 channels] (bf16; a vector is 8
-// consecutive channels), boxes of 136 tokens x several vectors.
+// consecutive channels), boxes of 136 tokens x several vectors; of z and y as [b][L][channels],
+// boxes of 64 channels x 128 tokens with 128-byte swizzling.
 struct WsMaps {
-    CUtensorMap x, B, C;
+    CUtensorMap x, B, C, z, y;
 };
 
 template <int R, bool SPLIT>
@@ -187,12 +189,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lo::OFF_TSLOT);
 
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t aC = s_base + Lo::OFF_C, aB = s_base + Lo::OFF_B, aM = s_base + Lo::OFF_M;
+    const uint32_t aC = s_base + Lo::OFF_C, aB = s_base + Lo::OFF_B, aZ = s_base + Lo::OFF_Z, aY = s_base + Lo::OFF_Y;
     const uint32_t aX = s_base + Lo::OFF_X, aXW = s_base + Lo::OFF_XW, aH = s_base + Lo::OFF_H;
     const uint32_t bar0 = smem_u32(&bars[0]), bar1 = smem_u32(&bars[1]), barX = smem_u32(&bars[2]);
     const uint32_t barP = smem_u32(&bars[3]), barC = smem_u32(&bars[4]);
     const uint32_t barE2 = smem_u32(&bars[5]), barF2 = smem_u32(&bars[7]), barN3 = smem_u32(&bars[9]);
     const uint32_t barTB = smem_u32(&bars[12]), barTX = smem_u32(&bars[13]);   // raw B/C rows, raw x rows
+    const uint32_t barZ = smem_u32(&bars[14]);                                      // z tile
 
     auto staged_channel = [&](int c) -> int64_t {
         if (c < kP) return (int64_t)h * kP + c;
@@ -201,6 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     };
 
     // ---- set-up
+    // the swizzled TMA tiles need a 1024-byte aligned base; every CTA sees the same base, so
+    // all of them leave here together (before any barrier) if it is not
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0) atomicExch(p.status, 1);
+        return;
+    }
     if (blockIdx.x == 0 && tid == 0) *p.status = 0;
     for (int c = tid; c < SROW; c += kThreads) {
         const int64_t ch = staged_channel(c);
@@ -225,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         mbar_init(barN3 + 16, 1);
         mbar_init(barTB, 1);
         mbar_init(barTX, 1);
+        mbar_init(barZ, 1);
         fence_mbar_init();
         prefetch_tmap(&maps.x);
         prefetch_tmap(&maps.B);
@@ -261,12 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     bool ok = true;
 
     const int64_t nblk = (p.L + kT - 1) / kT;
-    const __nv_bfloat16* gx = (const __nv_bfloat16*)p.x;
-    const __nv_bfloat16* gB = (const __nv_bfloat16*)p.B;
-    const __nv_bfloat16* gC = (const __nv_bfloat16*)p.C;
-    const __nv_bfloat16* gz = (const __nv_bfloat16*)p.z;
     const __nv_bfloat16* gdt = (const __nv_bfloat16*)p.dt;
-    __nv_bfloat16* gy = (__nv_bfloat16*)p.y;
     constexpr uint32_t kSliceBytes = (uint32_t)NS * kT * 2;
     const uint32_t slice_off = (uint32_t)q * kSliceBytes;
     auto blen = [&](int64_t k) { return (int)min((int64_t)kT, p.L - k * kT); };
@@ -494,9 +499,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     } else {
         // =========================== consumer (warps 8..15) ===========================
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        // 32 output channels of one row: gated values, optionally scaled by the norm and weighted
-        auto store_y = [&](__nv_bfloat16* dst, const float* gv, float scale, bool norm) {
-            uint4* yo = reinterpret_cast<uint4*>(dst);
+        // byte offset of 16-byte chunk c of token row r in a swizzled z/y tile
+        auto zy_off = [](int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); };
+        auto load_z = [&](int64_t kb) {   // thread kProd
+            mbar_arrive_expect_tx(barZ, (uint32_t)kT * kP * 2);
+            tma_load_3d(aZ, &maps.z, h * kP, (int)(kb * kT), (int)bi, barZ);
+        };
+        // this thread's 32 output channels of token crow into the y tile, then (thread kProd,
+        // after every consumer thread) one TMA store of the block's [128 x 64] box; the tile is
+        // free again once the previous store has been read out (waited before the named barrier
+        // that precedes every call)
+        auto store_y = [&](int64_t kb, const float* gv, float scale, bool norm) {
+            unsigned char* ty = smem + Lo::OFF_Y;
             const float2* nw2 = reinterpret_cast<const float2*>(s_nw + chalf * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -506,7 +520,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     const float2 gg = make_float2(gv[8 * v + 2 * e], gv[8 * v + 2 * e + 1]);
                     w[e] = pack_f2(norm ? mul2(mul2(gg, splat2(scale)), nw2[4 * v + e]) : gg);
                 }
-                yo[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(ty + zy_off(crow, chalf * 4 + v)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_async_smem();
+            named_sync(kBarCons, kThreads - kProd);
+            if (tid == kProd) {
+                tma_store_3d(&maps.y, aY, h * kP, (int)(kb * kT), (int)bi);
+                bulk_commit();
             }
         };
         // group RMSNorm of block kb: every CTA's sums of squares, the gated values from TMEM
@@ -520,24 +540,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             float gv[32];
             tmem_ld32(tmem + lane_base + kColG + chalf * 32, gv);
             tmem_wait_ld();
-            if (crow < blen(kb))
-                store_y(gy + (bi * p.L + kb * kT + crow) * p.y_ld + (int64_t)h * kP + chalf * 32, gv, scale, true);
+            store_y(kb, gv, scale, true);
         };
+        if (nblk > 0 && tid == kProd) load_z(0);
         for (int64_t k = 0; k < nblk; ++k) {
             const int64_t t0 = k * kT;
             const int len = blen(k);
             const int sl = (int)(k & 1);
             const uint32_t par = (uint32_t)(k & 1);
-            // z of this block for the gate
-            uint4 zr[4];
-            if (crow < len) {
-                const uint4* zs = reinterpret_cast<const uint4*>(gz + (bi * p.L + t0 + crow) * p.z_ld + (int64_t)h * kP + chalf * 32);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) zr[v] = zs[v];
-            } else {
-#pragma unroll
-                for (int v = 0; v < 4; ++v) zr[v] = make_uint4(0, 0, 0, 0);
-            }
             if (ok && !mbar_wait_bounded(barP, par, kWaitLimit)) ok = false;
             if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
             fence_after_sync();
@@ -549,27 +559,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             const float* dlb = s_dl + sl * kT;
             const float* vb = s_v + sl * kT;
             const float lam_end = lamb[kT - 1];
-            // masked, decayed M (row crow, columns chalf*64 .. +64), bf16, K-major
+            // masked, decayed M (row crow, columns chalf*64 .. +64) as bf16 pairs into TMEM
             {
                 const int i = crow;
                 const float li = lamb[i];
                 const bool fac = li > -96.0f;
                 const float ui = ex2(li);
-                unsigned char* sM = smem + Lo::OFF_M;
-                float cbf[64];
-                tmem_ld32(tmem + lane_base + kColCB + chalf * 64, cbf);
-                tmem_ld32(tmem + lane_base + kColCB + chalf * 64 + 32, cbf + 32);
-                tmem_wait_ld();
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
-                    const float* cb = cbf + part * 32;
+                    float cb[32];
+                    tmem_ld32(tmem + lane_base + kColCB + chalf * 64 + part * 32, cb);
+                    tmem_wait_ld();
+                    uint32_t w[16];
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         const int j0 = chalf * 64 + part * 32 + v * 8;
-                        uint32_t w[4];
                         if (j0 > i) {                 // above the diagonal: all zero
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) w[e] = 0u;
+                            for (int e = 0; e < 4; ++e) w[4 * v + e] = 0u;
                         } else if (fac) {
                             const float2* v2 = reinterpret_cast<const float2*>(vb + j0);
 #pragma unroll
@@ -577,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                                 float2 m = mul2(make_float2(cb[v * 8 + 2 * e], cb[v * 8 + 2 * e + 1]), mul2(splat2(ui), v2[e]));
                                 if (j0 + 2 * e > i) m.x = 0.0f;
                                 if (j0 + 2 * e + 1 > i) m.y = 0.0f;
-                                w[e] = pack_f2(m);
+                                w[4 * v + e] = pack_f2(m);
                             }
                         } else {
 #pragma unroll
@@ -585,12 +592,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                                 const int j = j0 + 2 * e;
                                 const float mx = (j <= i) ? cb[v * 8 + 2 * e] * ex2(li - lamb[j]) * dlb[j] : 0.0f;
                                 const float my = (j + 1 <= i) ? cb[v * 8 + 2 * e + 1] * ex2(li - lamb[j + 1]) * dlb[j + 1] : 0.0f;
-                                w[e] = pack_bf16x2(mx, my);
+                                w[4 * v + e] = pack_bf16x2(mx, my);
                             }
                         }
-                        const uint4 u = make_uint4(w[0], w[1], w[2], w[3]);
-                        *reinterpret_cast<uint4*>(sM + canon_off(i, chalf * 64 + part * 32 + v * 8, kT)) = u;
                     }
+                    tmem_st16(tmem + lane_base + kColM + chalf * 32 + part * 16, w);
                 }
             }
             // state update H <- exp(lam_end) H + S and its bf16 copy for the next block
@@ -614,8 +620,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     *reinterpret_cast<uint4*>(sH + canon_off(crow, chalf * 32 + 8 * v, kP)) = u;
                 }
             }
+            tmem_wait_st();
             fence_async_smem();
             fence_before_sync();
+            if (tid == kProd) bulk_wait_read_all();   // the previous y store has left the y tile
             named_sync(kBarCons, kThreads - kProd);
             if (tid == kProd) {
                 mbar_arrive_local(barC);   // C'B'^T and S^T read, H^T of block k+1 written
@@ -624,13 +632,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 const uint32_t aXs = aX + 16384 * (uint32_t)sl;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tmem + kColYi, sdesc(aM + kk * 256, 128, 2048), sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
+                    mma_bf16_ts(tmem + kColYi, tmem + kColM + kk * 8, sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
                 mma_commit(bar1);
             }
             if constexpr (!SPLIT) {
                 if (k >= 1) finish_norm(k - 1);   // overlaps the MMA M x' of this block
             }
             if (ok && !mbar_wait_bounded(bar1, par, kWaitLimit)) ok = false;
+            if (ok && !mbar_wait_bounded(barZ, par, kWaitLimit)) ok = false;
             fence_after_sync();
             // epilogue: y = Yi + exp(lam_i) Ys + D x', gate
             float gt[32];
@@ -642,16 +651,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 tmem_wait_ld();
                 const float2 el = splat2(ex2(lamb[i])), d2 = splat2(Dh);
                 const unsigned char* sX = smem + Lo::OFF_X + sl * 16384;
+                const unsigned char* tz = smem + Lo::OFF_Z;
                 float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     const uint4 xw = *reinterpret_cast<const uint4*>(sX + canon_off(i, chalf * 32 + 8 * v, kP));
+                    const uint4 zv = *reinterpret_cast<const uint4*>(tz + zy_off(i, chalf * 4 + v));
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c = 8 * v + 2 * e;
                         float2 y = fma2(el, make_float2(ys[c], ys[c + 1]), make_float2(yi[c], yi[c + 1]));
                         y = fma2(d2, bf2_to_f2((&xw.x)[e]), y);
-                        const float2 gg = mul2(y, silu2(bf2_to_f2((&zr[v].x)[e])));
+                        const float2 gg = mul2(y, silu2(bf2_to_f2((&zv.x)[e])));
                         gt[c] = gg.x;
                         gt[c + 1] = gg.y;
                         ss2 = fma2(gg, gg, ss2);
@@ -671,15 +682,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 }
             }
             fence_before_sync();
-            named_sync(kBarCons, kThreads - kProd);
-            if (tid == kProd) mbar_arrive_local(barE2 + 8 * sl);   // x'[sl] and the cumsum slot are free
             if constexpr (SPLIT) {
-                if (crow < len) store_y(gy + (bi * p.L + t0 + crow) * p.y_ld + (int64_t)h * kP + chalf * 32, gt, 1.0f, false);
+                if (tid == kProd) bulk_wait_read_all();
             }
+            named_sync(kBarCons, kThreads - kProd);
+            if (tid == kProd) {
+                mbar_arrive_local(barE2 + 8 * sl);   // x'[sl] and the cumsum slot are free
+                if (k + 1 < nblk) load_z(k + 1);     // the z tile is free
+            }
+            if constexpr (SPLIT) store_y(k, gt, 1.0f, false);
         }
         if constexpr (!SPLIT) {
-            if (nblk >= 1) finish_norm(nblk - 1);
+            if (nblk >= 1) {
+                if (tid == kProd) bulk_wait_read_all();
+                named_sync(kBarCons, kThreads - kProd);
+                finish_norm(nblk - 1);
+            }
         }
+        if (tid == kProd) bulk_wait_all();   // the y stores have completed
         // final SSM state of this head
         float* fs = p.final_ssm + (bi * p.H + h) * (int64_t)kP * kN;
 #pragma unroll
@@ -754,6 +774,21 @@ bool encode_rows(CUtensorMap* m, const void* base, int64_t width, int64_t ld, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [b][L][width] bf16 rows of `ld` elements; boxes of 64 channels x 128 tokens x 1 sequence,
+// 128-byte swizzled in shared memory.
+bool encode_tile(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b)
+{
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)L, (cuuint64_t)b};
+    const cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(L * ld * 2)};
+    const cuuint32_t box[3] = {(cuuint32_t)kP, (cuuint32_t)kT, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int R, bool SPLIT>
 cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
 {
@@ -763,7 +798,8 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     if (p.L > 0) {   // no block, no load: the maps stay unused
         if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, p.L, p.b, kP / 8) ||
             !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, p.L, p.b, Lo::NS / 8) ||
-            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, p.L, p.b, Lo::NS / 8))
+            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, p.L, p.b, Lo::NS / 8) ||
+            !encode_tile(&maps.z, p.z, p.HP(), p.z_ld, p.L, p.b) || !encode_tile(&maps.y, p.y, p.HP(), p.y_ld, p.L, p.b))
             return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
