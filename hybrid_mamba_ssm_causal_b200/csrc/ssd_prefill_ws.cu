@@ -25,8 +25,10 @@
 //   barP   producer: softplus/cumsum and x' of a block are in shared memory
 //   barC   consumer: C'B'^T and S^T read from TMEM, H^T of the next block written
 //   barE2  consumer: a block's x' and cumsum buffers are free again (2 slots by parity)
-//   barF2  every CTA of the cluster: its MMA1-3 of a block are done, so its B'/C' may be
-//          overwritten (2 slots; one arrival per CTA, multicast by its tensor-core commit)
+//   barF2  every CTA of the cluster: its MMA1-3 of a block are done (2 slots; one arrival per
+//          CTA, multicast by its tensor-core commit). Once all have arrived, no CTA reads its
+//          B'/C' of that block any more and every slice copy of it has landed, so the next
+//          block's slice may be written and sent.
 //   barN3  the sums of squares of a block from every CTA of the cluster have landed
 //          (st.async transaction bytes; 3 slots)
 // Barriers waited two blocks back use two slots, so a waiter never meets a barrier that
@@ -118,20 +120,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t mbar, uint32_t parity
         if (ok) return true;
         if (clock64() - t0 > limit) return false;
     }
-}
-
-// Non-blocking test of a barrier phase, acquiring at cluster scope when it has completed.
-__device__ __forceinline__ bool mbar_test_cluster(uint32_t mbar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(mbar), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 
 // Inclusive scan over the 128 threads of warps 4..7 (named barrier kBarScan).
@@ -339,9 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             const int len = blen(k);
             const int sl = (int)(k & 1);
             // buffers of this block: x'[sl] was last read by the consumer in block k-2, B'/C'/x'w
-            // by this CTA's MMAs of block k-1; the cumsum of this block is already in its slot
+            // by the MMAs of block k-1. Every CTA of the cluster has finished those: this CTA's
+            // B'/C' are no longer read, its own copies of block k-1's slice have landed in every
+            // peer (a peer's MMAs start only once they have), and every peer's B'/C' may take
+            // this block's slice. The cumsum of this block is already in its slot.
             if (tid == 0) {
-                if (k >= 1 && ok && !mbar_wait_bounded(bar0, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
+                if (k >= 1 && ok &&
+                    !mbar_wait_cluster(barF2 + 8 * (uint32_t)((k - 1) & 1), (uint32_t)(((k - 1) >> 1) & 1), kWaitLimit))
+                    ok = false;
                 if (k >= 2 && ok && !mbar_wait_bounded(barE2 + 8 * sl, (uint32_t)(((k - 2) >> 1) & 1), kWaitLimit)) ok = false;
                 mbar_arrive_expect_tx(barX, (uint32_t)(R - 1) * 2 * kSliceBytes);
             }
@@ -422,35 +415,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             conv_vectors(std::integral_constant<int, kVX>{}, std::integral_constant<int, kVBC>{});
             fence_async_smem();
             named_sync(kBarProd, kProd);
-            // this CTA's slice of B'/C' to every peer (warp 0, one copy per lane), once the peers'
-            // MMAs of block k-1 no longer read their B'/C': now if that is already so, else after
-            // the x' conv; and (lane 0) the next block's raw B/C rows, now that these are consumed
-            const int lane = tid & 31;
-            auto send_slice = [&]() {
-                if (lane >= 1 && lane <= 2 * (R - 1)) {
-                    const int idx = lane - 1;
+            // one duty per warp (lane 0), so that none lags the x' conv by more than one TMA or
+            // bulk-copy issue: warp 1 refills the raw B/C rows (these are consumed), warps 2.. each
+            // send one copy of this CTA's slice of B'/C' to a peer
+            if ((tid & 31) == 0) {
+                if (warp == 1) {
+                    if (k + 1 < nblk) load_bc(k + 1);
+                } else if (warp >= 2 && warp - 2 < 2 * (R - 1)) {
+                    const int idx = warp - 2;
                     const uint32_t rr = (uint32_t)((q + 1 + idx / 2) % R);
                     const uint32_t src = (idx & 1 ? aC : aB) + slice_off;
                     bulk_copy_to_peer(cluster_map(src, rr), src, kSliceBytes, cluster_map(barX, rr));
                 }
-            };
-            const uint32_t barF_prev = barF2 + 8 * (uint32_t)((k - 1) & 1), parF_prev = (uint32_t)(((k - 1) >> 1) & 1);
-            bool sent = false;
-            if (warp == 0) {
-                if (tid == 0 && k + 1 < nblk) load_bc(k + 1);
-                sent = __shfl_sync(0xffffffffu, (int)(k == 0 || (lane == 0 && mbar_test_cluster(barF_prev, parF_prev))), 0) != 0;
-                if (sent) send_slice();
             }
             // this block's raw x rows (the next block's B/C rows may be in flight)
             if (ok && !mbar_wait_bounded(barTX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
             conv_vectors(std::integral_constant<int, 0>{}, std::integral_constant<int, kVX>{});
             fence_async_smem();
             named_sync(kBarProd, kProd);
-            if (warp == 0 && !sent) {
-                if (tid == 0 && ok && !mbar_wait_cluster(barF_prev, parF_prev, kWaitLimit)) ok = false;
-                __syncwarp();
-                send_slice();
-            }
             if (tid == 0) {
                 if (ok && !mbar_wait_bounded(barX, (uint32_t)(k & 1), kWaitLimit)) ok = false;
                 // the consumer has read C'B'^T and S^T of block k-1 and written H^T for this block
@@ -626,7 +608,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             if (tid == kProd) bulk_wait_read_all();   // the previous y store has left the y tile
             named_sync(kBarCons, kThreads - kProd);
             if (tid == kProd) {
-                mbar_arrive_local(barC);   // C'B'^T and S^T read, H^T of block k+1 written
                 fence_after_sync();
                 const uint32_t id_yi = idesc_bf16(128, 64, 0, 1);
                 const uint32_t aXs = aX + 16384 * (uint32_t)sl;
@@ -634,6 +615,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16_ts(tmem + kColYi, tmem + kColM + kk * 8, sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
                 mma_commit(bar1);
+                // C'B'^T and S^T read, H^T of block k+1 written; the producer's next MMAs queue
+                // behind M x'
+                mbar_arrive_local(barC);
             }
             if constexpr (!SPLIT) {
                 if (k >= 1) finish_norm(k - 1);   // overlaps the MMA M x' of this block
