@@ -116,6 +116,43 @@ def kernel_bytes(name, w, batch, seqlen) -> int | None:
     return None
 
 
+# ------------------------------------------------------------------ measured DRAM traffic
+
+KERNEL_SOURCES = {"tc_prefill": ["hybrid_mamba_ssm_causal_b200/csrc/ssd_prefill_ws.cu",
+                                 "hybrid_mamba_ssm_causal_b200/csrc/ssd_tc_util.cuh"],
+                  "decode_step": ["hybrid_mamba_ssm_causal_b200/csrc/ssd_decode.cu"]}
+TRAFFIC_SUMMARIES = {"tc_prefill": "profiles/ssd_prefill_ws_small_bf16.md",
+                     "decode_step": "profiles/decode_step_decode_bf16.md"}
+
+
+def sources_sha256(name: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[name]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(name: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch from the committed ncu summary
+    of this kernel, or None when there is none or the kernel's sources changed since."""
+    if name not in TRAFFIC_SUMMARIES:
+        return None
+    try:
+        with open(os.path.join(ROOT, TRAFFIC_SUMMARIES[name])) as f:
+            kv = dict(line.split(":", 1) for line in f.read().splitlines()
+                      if line.startswith(("traffic_bytes_per_launch:", "kernel_sources_sha256:")))
+    except OSError:
+        return None
+    if kv.get("kernel_sources_sha256", "").strip() != sources_sha256(name):
+        return None
+    try:
+        return float(kv["traffic_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------------ clocks
 
 class Clocks:
@@ -338,7 +375,7 @@ def main():
         avg_ms = tot_ms / n
         ach = kb / (avg_ms * 1e-3) / 1e9 if kb else None
         roofline = {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                    "frac": (ach / hbm) if ach else None, "traffic": None, "peak_source": peak_src,
+                    "frac": (ach / hbm) if ach else None, "traffic": measured_traffic(name), "peak_source": peak_src,
                     "avg_launch_us": avg_ms * 1e3, "algorithmic_bytes_per_launch": kb,
                     "share_of_step": tot_ms / (ms_local * a.steps)}
 
@@ -414,7 +451,8 @@ def main():
                   "value": world / (dms * 1e-3), "unit": "steps/s", "tokens_per_s": world * wd.batch / (dms * 1e-3),
                   "us_per_step": dms * 1e3,
                   "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                               "frac": ach / hbm, "algorithmic_bytes_per_launch": db, "peak_source": peak_src}}
+                               "frac": ach / hbm, "traffic": measured_traffic("decode_step"),
+                               "algorithmic_bytes_per_launch": db, "peak_source": peak_src}}
 
     ck = clocks.stop()   # sampled over the prefill, end-to-end and decode timed regions
     cpu = None
