@@ -10,16 +10,18 @@ namespace ssd {
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
-                                         int act)
+WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int H, int P, int G, int N,
+                                         int Q, int act)
 {
     WorkspaceLayout w{};
     if (prefill_tc_supported(act, P, N, H, G)) {   // everything stays on chip
         w.status = 0;
-        w.xbc = w.delta = w.lam = w.states = w.ypre = w.ssp = 256;
+        w.xbc = w.delta = w.lam = w.states = w.ypre = w.ssp = w.bc_conv = 256;
         w.total = 256;
-        if (prefill_tc_split(H, G))
-            w.total = align256(256 + (size_t)(b * L * H) * (size_t)prefill_ws_partials_per_head() * 4);
+        if (prefill_tc_split(H, G)) {
+            w.bc_conv = align256(256 + (size_t)(rows * H) * (size_t)prefill_ws_partials_per_head() * 4);
+            w.total = align256(w.bc_conv + (size_t)(b * 2 * G * N) * 3 * 2);
+        }
         return w;
     }
     const size_t es = act == SSD_BF16 ? 2 : 4;
@@ -32,7 +34,7 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int
     w.lam = off;    off = align256(off + (size_t)(b * H * L) * 4);
     w.states = off; off = align256(off + (size_t)(b * nc * H) * (size_t)P * N * 4);
     w.ypre = off;   off = align256(off + (size_t)(b * L * HP) * 4);
-    w.ssp = off;
+    w.ssp = w.bc_conv = off;
     w.total = off;
     return w;
 }
@@ -88,8 +90,8 @@ extern "C" {
 size_t ssd_mixer_prefill_workspace_size(const ssd_dims* d)
 {
     if (check_dims(d, false) != SSD_OK) return 0;
-    return ssd::prefill_workspace_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->ngroups,
-                                         d->dstate, d->chunk, d->act)
+    return ssd::prefill_workspace_layout(d->batch, d->seqlen, d->batch * d->seqlen, d->nheads, d->headdim,
+                                         d->ngroups, d->dstate, d->chunk, d->act)
         .total;
 }
 
@@ -113,8 +115,8 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
         return SSD_ERR_UNSUPPORTED;
     if ((init_conv_state && ((uintptr_t)init_conv_state % es)) || ((uintptr_t)final_conv_state % es))
         return SSD_ERR_UNSUPPORTED;
-    const ssd::WorkspaceLayout wl = ssd::prefill_workspace_layout(
-        d->batch, d->seqlen, d->nheads, d->headdim, d->ngroups, d->dstate, d->chunk, d->act);
+    const ssd::WorkspaceLayout wl = ssd::prefill_workspace_layout(d->batch, d->seqlen, d->batch * d->seqlen, d->nheads,
+                                                                  d->headdim, d->ngroups, d->dstate, d->chunk, d->act);
     if (!workspace || workspace_bytes < wl.total || ((uintptr_t)workspace & 255u))
         return SSD_ERR_INVALID_ARG;
     if (d->seqlen > 0 && d->batch > 0) {
@@ -142,10 +144,72 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.states = (float*)(ws + wl.states);
     p.ypre = (float*)(ws + wl.ypre);
     p.ssp = (float*)(ws + wl.ssp);
+    p.bc_conv = ws + wl.bc_conv;
     cudaStream_t st = (cudaStream_t)stream;
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
     if ((tc ? ssd::launch_prefill_ws(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
         return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+size_t ssd_mixer_prefill_varlen_workspace_size(const ssd_dims* d)
+{
+    if (check_dims(d, false) != SSD_OK ||
+        !ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups))
+        return 0;
+    return ssd::prefill_workspace_layout(d->batch, d->seqlen, d->seqlen, d->nheads, d->headdim, d->ngroups,
+                                         d->dstate, d->chunk, d->act)
+        .total;
+}
+
+ssd_status ssd_mixer_prefill_varlen(const ssd_dims* d, const int32_t* cu_seqlens, const int32_t* slot_idx,
+                                    const uint8_t* has_init, const void* x, int64_t x_ld, const void* z,
+                                    int64_t z_ld, const void* B, int64_t B_ld, const void* C, int64_t C_ld,
+                                    const void* dt, int64_t dt_ld, const float* A, const float* D,
+                                    const float* conv_w, const float* conv_b, const float* dt_bias,
+                                    const float* norm_w, float* ssm_state, void* conv_state, void* y,
+                                    int64_t y_ld, void* workspace, size_t workspace_bytes, void* stream)
+{
+    const ssd_status ds = check_dims(d, false);
+    if (ds != SSD_OK) return ds;
+    if (!ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups))
+        return SSD_ERR_UNSUPPORTED;
+    if (d->seqlen > 0x7fffff00LL) return SSD_ERR_UNSUPPORTED;   // token rows are int32 (cu_seqlens)
+    const size_t es = 2;
+    const int64_t HP = (int64_t)d->nheads * d->headdim, GN = (int64_t)d->ngroups * d->dstate;
+    if (!A || !D || !conv_w || !conv_b || !dt_bias || !norm_w || !ssm_state || !conv_state || !cu_seqlens)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(conv_w) || !aligned16(ssm_state) || ((uintptr_t)conv_state % es) ||
+        ((uintptr_t)cu_seqlens & 3u) || (slot_idx && ((uintptr_t)slot_idx & 3u)))
+        return SSD_ERR_UNSUPPORTED;
+    const ssd::WorkspaceLayout wl = ssd::prefill_workspace_layout(d->batch, d->seqlen, d->seqlen, d->nheads,
+                                                                  d->headdim, d->ngroups, d->dstate, d->chunk, d->act);
+    if (!workspace || workspace_bytes < wl.total || ((uintptr_t)workspace & 255u)) return SSD_ERR_INVALID_ARG;
+    if (d->seqlen > 0) {
+        if (!x || !z || !B || !C || !dt || !y) return SSD_ERR_INVALID_ARG;
+        if (!row_ok(x, x_ld, HP, es, true) || !row_ok(z, z_ld, HP, es, true) ||
+            !row_ok(B, B_ld, GN, es, true) || !row_ok(C, C_ld, GN, es, true) ||
+            !row_ok(y, y_ld, HP, es, true) || !row_ok(dt, dt_ld, d->nheads, es, false))
+            return SSD_ERR_UNSUPPORTED;
+    }
+    if (d->batch == 0) return SSD_OK;
+    ssd::PrefillParams p{};
+    p.b = d->batch; p.L = d->seqlen;
+    p.H = d->nheads; p.P = d->headdim; p.G = d->ngroups; p.N = d->dstate; p.K = d->dconv;
+    p.Q = d->chunk; p.eps = d->eps; p.act = d->act;
+    p.nc = (p.L + p.Q - 1) / p.Q;
+    p.x = x; p.z = z; p.B = B; p.C = C; p.dt = dt;
+    p.x_ld = x_ld; p.z_ld = z_ld; p.B_ld = B_ld; p.C_ld = C_ld; p.dt_ld = dt_ld;
+    p.A = A; p.D = D; p.conv_w = conv_w; p.conv_b = conv_b; p.dt_bias = dt_bias; p.norm_w = norm_w;
+    p.init_ssm = ssm_state; p.init_conv = conv_state;
+    p.final_ssm = ssm_state; p.final_conv = conv_state;
+    p.y = y; p.y_ld = y_ld;
+    p.cu_seqlens = cu_seqlens; p.slot_idx = slot_idx; p.has_init = has_init;
+    char* ws = (char*)workspace;
+    p.status = (int*)(ws + wl.status);
+    p.ssp = (float*)(ws + wl.ssp);
+    p.bc_conv = ws + wl.bc_conv;
+    if (ssd::launch_prefill_ws(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }
 

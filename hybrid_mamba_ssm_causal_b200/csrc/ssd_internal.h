@@ -36,11 +36,21 @@ struct PrefillParams {
     float* lam;      // [b][H][L] within-chunk inclusive cumsum of delta*A
     float* states;   // [b][nc][H][P][N] chunk states, then states entering each chunk
     float* ypre;     // [b][L][HP] y before the gate and norm
-    float* ssp;      // tensor-core path, groups wider than one cluster: [b][L][H][parts] sums of g^2
+    float* ssp;      // tensor-core path, groups wider than one cluster: [rows][H][parts] sums of g^2
+    void* bc_conv;   // tensor-core path, groups wider than one cluster: [b][2 GN][K-1] final B/C
+                     // conv state, staged until every cluster of the group has read the initial one
+    // Packed variable-length sequences on state slots (cu_seqlens != nullptr): b sequences,
+    // L = total packed tokens, sequence i owns rows cu_seqlens[i] .. cu_seqlens[i+1]-1; its
+    // states are the slot slot_idx[i] (identity when null) of init_ssm/init_conv, which
+    // alias final_ssm/final_conv; has_init[i] == 0 starts it from zero states.
+    const int32_t* cu_seqlens;
+    const int32_t* slot_idx;
+    const uint8_t* has_init;
 
     SSD_HD int64_t HP() const { return (int64_t)H * P; }
     SSD_HD int64_t GN() const { return (int64_t)G * N; }
     SSD_HD int64_t Cc() const { return HP() + 2 * GN(); }
+    SSD_HD int64_t rows() const { return cu_seqlens ? L : b * L; }   // token rows of x, z, y, ...
 };
 
 struct DecodeParams {
@@ -64,10 +74,11 @@ struct DecodeParams {
 
 // Workspace layout of one prefill call; offsets in bytes, each 256-byte aligned.
 struct WorkspaceLayout {
-    size_t status, xbc, delta, lam, states, ypre, ssp, total;
+    size_t status, xbc, delta, lam, states, ypre, ssp, bc_conv, total;
 };
-WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q,
-                                         int act);
+// rows = token rows of one call (b*L, or the packed total of a variable-length call).
+WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int H, int P, int G, int N,
+                                         int Q, int act);
 
 // Tensor-core path (ssd_prefill_ws.cu): bf16 activations, P = 64, N = 128, 2 or a multiple
 // of 4 heads per group. It keeps every intermediate on chip; the workspace holds only the

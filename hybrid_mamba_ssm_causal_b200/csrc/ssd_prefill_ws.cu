@@ -162,6 +162,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const int h = g * rpg + (int)(cid % ncl) * R + q;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int64_t HP = p.HP(), GN = p.GN(), Cc = p.Cc();
+    // this CTA's sequence: its first token row, length, state slot, and whether it starts from
+    // the states given (packed variable-length calls read them from their slot arrays)
+    const bool varlen = p.cu_seqlens != nullptr;
+    const int64_t row0 = varlen ? (int64_t)p.cu_seqlens[bi] : bi * p.L;
+    const int64_t seqlen = varlen ? (int64_t)p.cu_seqlens[bi + 1] - row0 : p.L;
+    const int64_t sidx = varlen && p.slot_idx ? (int64_t)p.slot_idx[bi] : bi;
+    const bool cont = varlen ? (!p.has_init || p.has_init[bi] != 0) : true;
+    const bool init_ssm = cont && p.init_ssm != nullptr, init_conv = cont && p.init_conv != nullptr;
+    // coordinates of token 0 in the tensor maps (token, sequence)
+    const int tmap_t0 = varlen ? (int)row0 : 0, tmap_b = varlen ? 0 : (int)bi;
 
     float* mf = reinterpret_cast<float*>(smem + Lo::OFF_MISC);
     float* s_lam = mf + Lo::F_LAM;
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const int crow = tid & 127, chalf = (tid - kProd) >> 7;   // consumer row and column half
     float H[32];
     if (consumer) {
-        const float* h0 = p.init_ssm ? p.init_ssm + (bi * p.H + h) * (int64_t)kP * kN : nullptr;
+        const float* h0 = init_ssm ? p.init_ssm + (sidx * p.H + h) * (int64_t)kP * kN : nullptr;
 #pragma unroll
         for (int i = 0; i < 32; ++i) H[i] = h0 ? h0[(int64_t)(chalf * 32 + i) * kN + crow] : 0.0f;
         unsigned char* sH = smem + Lo::OFF_H;
@@ -258,11 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const float bias = p.dt_bias[h];
     bool ok = true;
 
-    const int64_t nblk = (p.L + kT - 1) / kT;
+    const int64_t nblk = (seqlen + kT - 1) / kT;
     const __nv_bfloat16* gdt = (const __nv_bfloat16*)p.dt;
     constexpr uint32_t kSliceBytes = (uint32_t)NS * kT * 2;
     const uint32_t slice_off = (uint32_t)q * kSliceBytes;
-    auto blen = [&](int64_t k) { return (int)min((int64_t)kT, p.L - k * kT); };
+    auto blen = [&](int64_t k) { return (int)min((int64_t)kT, seqlen - k * kT); };
 
     if (!consumer) {
         // =========================== producer (warps 0..7) ===========================
@@ -271,13 +281,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         // each for this CTA's B and C vectors on barTB; rows outside the sequence read as zeros
         auto load_bc = [&](int64_t kb) {
             mbar_arrive_expect_tx(barTB, (uint32_t)kVBC * kStageRows * 16);
-            const int t0 = (int)(kb * kT) - kStageTok, vb = (g * kN + q * NS) / 8;
-            tma_load_4d(smem_u32(stage + kVX * kStageRows), &maps.B, 0, t0, vb, (int)bi, barTB);
-            tma_load_4d(smem_u32(stage + (kVX + NS / 8) * kStageRows), &maps.C, 0, t0, vb, (int)bi, barTB);
+            const int t0 = tmap_t0 + (int)(kb * kT) - kStageTok, vb = (g * kN + q * NS) / 8;
+            tma_load_4d(smem_u32(stage + kVX * kStageRows), &maps.B, 0, t0, vb, tmap_b, barTB);
+            tma_load_4d(smem_u32(stage + (kVX + NS / 8) * kStageRows), &maps.C, 0, t0, vb, tmap_b, barTB);
         };
         auto load_x = [&](int64_t kb) {
             mbar_arrive_expect_tx(barTX, (uint32_t)kVX * kStageRows * 16);
-            tma_load_4d(smem_u32(stage), &maps.x, 0, (int)(kb * kT) - kStageTok, h * kVX, (int)bi, barTX);
+            tma_load_4d(smem_u32(stage), &maps.x, 0, tmap_t0 + (int)(kb * kT) - kStageTok, h * kVX, tmap_b, barTX);
         };
         // softplus and cumsum of block kb into its slot (warps 4..7, token tid - 128), then dt of
         // block kb + 1, a whole block ahead of its use
@@ -290,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 dl = softplus(dt_next + bias);
                 a2 = dl * A2;
             }
-            if (kb + 1 < nblk && (kb + 1) * kT + tok < p.L)
-                dt_next = __bfloat162float(gdt[(bi * p.L + (kb + 1) * kT + tok) * p.dt_ld + h]);
+            if (kb + 1 < nblk && (kb + 1) * kT + tok < seqlen)
+                dt_next = __bfloat162float(gdt[(row0 + (kb + 1) * kT + tok) * p.dt_ld + h]);
             const float lam = scan128(a2, s_scan);
             s_lam[slb * kT + tok] = lam;
             s_dl[slb * kT + tok] = dl;
@@ -305,13 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 load_x(0);
             }
             if (warp >= 4) {
-                if (tok < p.L) dt_next = __bfloat162float(gdt[(bi * p.L + tok) * p.dt_ld + h]);
+                if (tok < seqlen) dt_next = __bfloat162float(gdt[(row0 + tok) * p.dt_ld + h]);
                 scan_block(0);
             }
         }
         // the three rows before the sequence hold the initial conv state (zeros without one), not
-        // the TMA's fill: written once block 0's rows have landed
-        if (nblk == 0 || p.init_conv) {
+        // the TMA's fill or a neighbouring packed sequence: written once block 0's rows have landed
+        if (nblk == 0 || init_conv || varlen) {
             if (nblk > 0) {
                 if (ok && !mbar_wait_bounded(barTB, 0, kWaitLimit)) ok = false;
                 if (ok && !mbar_wait_bounded(barTX, 0, kWaitLimit)) ok = false;
@@ -319,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             for (int e = tid; e < 3 * SROW; e += kProd) {
                 const int kk = e / SROW, c = e % SROW;
                 __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
-                if (p.init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(bi * Cc + staged_channel(c)) * 3 + kk];
+                if (init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(sidx * Cc + staged_channel(c)) * 3 + kk];
                 reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + kk)[c % 8] = v;
             }
         }
@@ -473,10 +483,21 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         // final conv state: the last three raw inputs of the staged channels
         const int len_last = nblk > 0 ? blen(nblk - 1) : 0;
         named_sync(kBarProd, kProd);
+        // B/C channels of a group wider than one cluster: several clusters hold the same values
+        // and may run at different times, so the first cluster of the group stages them and a
+        // later kernel writes them out (an in-place final state must not be overwritten before
+        // every cluster has read it as its initial state)
+        const bool first_cluster = (cid % ncl) == 0;
         for (int e = tid; e < 3 * SROW; e += kProd) {
             const int kk = e / SROW, c = e % SROW;
-            ((__nv_bfloat16*)p.final_conv)[(bi * Cc + staged_channel(c)) * 3 + kk] =
+            const __nv_bfloat16 v =
                 reinterpret_cast<const __nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + len_last + kk)[c % 8];
+            if (SPLIT && c >= kP) {
+                if (first_cluster)
+                    ((__nv_bfloat16*)p.bc_conv)[(bi * 2 * GN + staged_channel(c) - HP) * 3 + kk] = v;
+            } else {
+                ((__nv_bfloat16*)p.final_conv)[(sidx * Cc + staged_channel(c)) * 3 + kk] = v;
+            }
         }
     } else {
         // =========================== consumer (warps 8..15) ===========================
@@ -485,14 +506,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         auto zy_off = [](int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); };
         auto load_z = [&](int64_t kb) {   // thread kProd
             mbar_arrive_expect_tx(barZ, (uint32_t)kT * kP * 2);
-            tma_load_3d(aZ, &maps.z, h * kP, (int)(kb * kT), (int)bi, barZ);
+            tma_load_3d(aZ, &maps.z, h * kP, tmap_t0 + (int)(kb * kT), tmap_b, barZ);
         };
         // this thread's 32 output channels of token crow into the y tile, then (thread kProd,
         // after every consumer thread) one TMA store of the block's [128 x 64] box; the tile is
         // free again once the previous store has been read out (waited before the named barrier
         // that precedes every call)
+        // The last, shorter block of a packed sequence is stored row by row instead: a box would
+        // also write the first rows of the next sequence.
         auto store_y = [&](int64_t kb, const float* gv, float scale, bool norm) {
+            const bool rows_only = varlen && blen(kb) < kT;
             unsigned char* ty = smem + Lo::OFF_Y;
+            uint4* yrow = reinterpret_cast<uint4*>((__nv_bfloat16*)p.y + (row0 + kb * kT + crow) * p.y_ld + h * kP + chalf * 32);
             const float2* nw2 = reinterpret_cast<const float2*>(s_nw + chalf * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -502,12 +527,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     const float2 gg = make_float2(gv[8 * v + 2 * e], gv[8 * v + 2 * e + 1]);
                     w[e] = pack_f2(norm ? mul2(mul2(gg, splat2(scale)), nw2[4 * v + e]) : gg);
                 }
-                *reinterpret_cast<uint4*>(ty + zy_off(crow, chalf * 4 + v)) = make_uint4(w[0], w[1], w[2], w[3]);
+                if (!rows_only) *reinterpret_cast<uint4*>(ty + zy_off(crow, chalf * 4 + v)) = make_uint4(w[0], w[1], w[2], w[3]);
+                else if (crow < blen(kb)) yrow[v] = make_uint4(w[0], w[1], w[2], w[3]);
             }
+            if (rows_only) return;
             fence_async_smem();
             named_sync(kBarCons, kThreads - kProd);
             if (tid == kProd) {
-                tma_store_3d(&maps.y, aY, h * kP, (int)(kb * kT), (int)bi);
+                tma_store_3d(&maps.y, aY, h * kP, tmap_t0 + (int)(kb * kT), tmap_b);
                 bulk_commit();
             }
         };
@@ -654,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 }
                 const float ss = ss2.x + ss2.y;
                 if constexpr (SPLIT) {
-                    if (i < len) p.ssp[((bi * p.L + t0 + i) * p.H + h) * 2 + chalf] = ss;
+                    if (i < len) p.ssp[((row0 + t0 + i) * p.H + h) * 2 + chalf] = ss;
                 } else {
                     const uint32_t nsl = (uint32_t)(k % 3);
                     const uint32_t dst = smem_u32(s_red + ((nsl * R + q) * 2 + chalf) * 128 + i);
@@ -685,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         }
         if (tid == kProd) bulk_wait_all();   // the y stores have completed
         // final SSM state of this head
-        float* fs = p.final_ssm + (bi * p.H + h) * (int64_t)kP * kN;
+        float* fs = p.final_ssm + (sidx * p.H + h) * (int64_t)kP * kN;
 #pragma unroll
         for (int i = 0; i < 32; ++i) fs[(int64_t)(chalf * 32 + i) * kN + crow] = H[i];
     }
@@ -702,7 +729,7 @@ __global__ void __launch_bounds__(256) ws_norm_finish_kernel(PrefillParams p)
 {
     const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (w >= p.b * p.L * p.G) return;
+    if (w >= p.rows() * p.G) return;
     const int64_t row = w / p.G;
     const int g = (int)(w % p.G);
     const int rpg = p.H / p.G, gs = rpg * kP;
@@ -773,17 +800,30 @@ bool encode_tile(CUtensorMap* m, const void* base, int64_t width, int64_t ld, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The staged B/C part of the final conv state, into each sequence's slot.
+__global__ void __launch_bounds__(256) ws_bc_conv_out_kernel(PrefillParams p)
+{
+    const int64_t per = 2 * p.GN() * 3;
+    const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (e >= p.b * per) return;
+    const int64_t bi = e / per, r = e % per;
+    const int64_t sidx = p.cu_seqlens && p.slot_idx ? (int64_t)p.slot_idx[bi] : bi;
+    ((__nv_bfloat16*)p.final_conv)[(sidx * p.Cc() + p.HP()) * 3 + r] = ((const __nv_bfloat16*)p.bc_conv)[e];
+}
+
 template <int R, bool SPLIT>
 cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
 {
     using Lo = WsLayout<R>;
     WsMaps maps;
     memset(&maps, 0, sizeof(maps));
+    // packed sequences: one row of all the packed tokens
+    const int64_t mL = p.L, mb = p.cu_seqlens ? 1 : p.b;
     if (p.L > 0) {   // no block, no load: the maps stay unused
-        if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, p.L, p.b, kP / 8) ||
-            !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, p.L, p.b, Lo::NS / 8) ||
-            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, p.L, p.b, Lo::NS / 8) ||
-            !encode_tile(&maps.z, p.z, p.HP(), p.z_ld, p.L, p.b) || !encode_tile(&maps.y, p.y, p.HP(), p.y_ld, p.L, p.b))
+        if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, mL, mb, kP / 8) ||
+            !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, mL, mb, Lo::NS / 8) ||
+            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, mL, mb, Lo::NS / 8) ||
+            !encode_tile(&maps.z, p.z, p.HP(), p.z_ld, mL, mb) || !encode_tile(&maps.y, p.y, p.HP(), p.y_ld, mL, mb))
             return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -806,10 +846,17 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
         e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT>, p, maps);
         if (e != cudaSuccess) return e;
     }
-    if (SPLIT && p.L > 0) {
+    if (SPLIT && p.rows() > 0) {
         LaunchScope ls("tc_norm_finish", st);
-        const int64_t warps = p.b * p.L * p.G;
+        const int64_t warps = p.rows() * p.G;
         ws_norm_finish_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (SPLIT) {
+        LaunchScope ls("tc_bc_conv_out", st);
+        const int64_t n = p.b * 2 * p.GN() * 3;
+        ws_bc_conv_out_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
         e = cudaGetLastError();
     }
     return e;

@@ -32,7 +32,7 @@ SSD_F32, SSD_BF16 = 0, 1
 SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_decode_step",
            "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version",
            "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read",
-           "ssd_mixer_prefill_static")
+           "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen")
 
 
 class SsdError(RuntimeError):
@@ -106,6 +106,11 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_prefill_static.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
                                              [FP, P, P, I64, FP, P, V])
     lib.ssd_mixer_prefill_static.restype = ctypes.c_int
+    lib.ssd_mixer_prefill_varlen_workspace_size.argtypes = [ctypes.POINTER(_CDims)]
+    lib.ssd_mixer_prefill_varlen_workspace_size.restype = ctypes.c_size_t
+    lib.ssd_mixer_prefill_varlen.argtypes = ([ctypes.POINTER(_CDims), P, P, P] + [P, I64] * 5 + [FP] * 6 +
+                                             [FP, P, P, I64, P, ctypes.c_size_t, V])
+    lib.ssd_mixer_prefill_varlen.restype = ctypes.c_int
     lib.ssd_mixer_workspace_status.argtypes = [P, V]
     lib.ssd_mixer_workspace_status.restype = ctypes.c_int
     lib.ssd_status_string.argtypes = [ctypes.c_int]
@@ -205,6 +210,38 @@ def ssd_mixer_prefill_static(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, d
         _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
         py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
         _stream(stream)))
+
+
+def ssd_mixer_prefill_varlen_workspace_size(dims: Dims) -> int:
+    cd = dims.c()
+    return int(load_library().ssd_mixer_prefill_varlen_workspace_size(ctypes.byref(cd)))
+
+
+def ssd_mixer_prefill_varlen(dims: Dims, cu_seqlens, slot_idx, has_init, x, z, B, C, dt, A, D, conv_w,
+                             conv_b, dt_bias, norm_w, ssm_state, conv_state, y, workspace,
+                             stream=None) -> None:
+    """Packed variable-length prefill on state slots: dims.batch sequences, dims.seqlen packed
+    tokens in total (x ... y are [T, width] row views); cu_seqlens int32 [b+1], slot_idx int32
+    [b] or None, has_init uint8 [b] or None, all on the device."""
+    lib = load_library()
+    rows = dims.seqlen
+    HP, GN = dims.d_inner, dims.ngroups * dims.dstate
+    if cu_seqlens.dtype != torch.int32 or (slot_idx is not None and slot_idx.dtype != torch.int32):
+        raise TypeError("cu_seqlens and slot_idx must be int32")
+    if has_init is not None and has_init.dtype != torch.uint8:
+        raise TypeError("has_init must be uint8")
+    args = []
+    for t, name, w in ((x, "x", HP), (z, "z", HP), (B, "B", GN), (C, "C", GN), (dt, "dt", dims.nheads)):
+        args += list(_rows(t, name, rows, w))
+    py, y_ld = _rows(y, "y", rows, HP)
+    cd = dims.c()
+    st = lib.ssd_mixer_prefill_varlen(
+        ctypes.byref(cd), _dev(cu_seqlens, "cu_seqlens"), _dev(slot_idx, "slot_idx"), _dev(has_init, "has_init"),
+        *args, _dev(A, "A"), _dev(D, "D"), _dev(conv_w, "conv_w"), _dev(conv_b, "conv_b"),
+        _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"), _dev(ssm_state, "ssm_state"),
+        _dev(conv_state, "conv_state"), py, y_ld, _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "ssd_mixer_prefill_varlen")
 
 
 def ssd_mixer_decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,

@@ -126,6 +126,51 @@ SSD_API ssd_status ssd_mixer_prefill(const ssd_dims* dims,
                              void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* Bytes of device workspace ssd_mixer_prefill_varlen needs for `dims` (dims->batch
+ * sequences, dims->seqlen packed tokens in total); 0 when the dims are invalid or the
+ * shape is one the packed entry point does not run. */
+SSD_API size_t ssd_mixer_prefill_varlen_workspace_size(const ssd_dims* dims);
+
+/* Prefill of packed variable-length sequences on state slots: b sequences of any
+ * lengths, their tokens back to back in one token dimension, each continuing from (or
+ * starting afresh on) the state slot it owns. This is the engine case of gllm PR #86,
+ * section "Validation": several sequences in one batch, each Mamba layer picking up the
+ * recurrent state of its own slot, of which one may be prefilling while another decodes
+ * (a one-token sequence here runs the same arithmetic as ssd_mixer_decode_step).
+ *
+ * dims->batch = b sequences; dims->seqlen = T, the total number of packed tokens;
+ * dims->chunk as for ssd_mixer_prefill.
+ * cu_seqlens [b+1] int32 (device): sequence i owns packed rows cu_seqlens[i] ..
+ *   cu_seqlens[i+1]-1, with cu_seqlens[0] = 0, non-decreasing, cu_seqlens[b] = T. A
+ *   length may be 0: the final states are then the initial ones (the slot's own, or
+ *   zeros where has_init is 0).
+ * slot_idx [b] int32 (device; NULL = sequence i uses slot i): distinct, in range.
+ * has_init [b] uint8 (device; NULL = all nonzero): nonzero = the sequence continues from
+ *   the states in its slot; 0 = it starts from zero states (a new prompt).
+ * x, z [T][HP]; B, C [T][GN]; dt [T][H]; y [T][HP]: packed rows with the strides given,
+ *   same alignment rules as ssd_mixer_prefill.
+ * ssm_state [nslots][H][P][N] fp32 and conv_state [nslots][Cc][K-1]: read as the initial
+ *   states where has_init says so, and overwritten in place with the final states.
+ * workspace: ssd_mixer_prefill_varlen_workspace_size(dims) bytes, 256-byte aligned.
+ * Runs the tensor-core kernel only: bf16 activations, P = 64, N = 128 and 2 or a multiple
+ * of 4 heads per group; other shapes return SSD_ERR_UNSUPPORTED. The library cannot check
+ * device-resident cu_seqlens, slot_idx or has_init. */
+SSD_API ssd_status ssd_mixer_prefill_varlen(const ssd_dims* dims,
+                                    const int32_t* cu_seqlens, const int32_t* slot_idx,
+                                    const uint8_t* has_init,
+                                    const void* x, int64_t x_ld,
+                                    const void* z, int64_t z_ld,
+                                    const void* B, int64_t B_ld,
+                                    const void* C, int64_t C_ld,
+                                    const void* dt, int64_t dt_ld,
+                                    const float* A, const float* D,
+                                    const float* conv_w, const float* conv_b,
+                                    const float* dt_bias, const float* norm_w,
+                                    float* ssm_state, void* conv_state,
+                                    void* y, int64_t y_ld,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 /* Decode step: advance b sequences by one token each, in place on their state
  * slots (the one-token-at-a-time decode of gllm PR #86, section "Validation", where
  * each Mamba layer picks up from the state held in the sequence's slot).

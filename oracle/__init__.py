@@ -194,6 +194,36 @@ def prefill_dict(d: Dims, inp: dict, **kw):
                    inp.get("init_ssm"), inp.get("init_conv"), **kw)
 
 
+def prefill_varlen(d: Dims, cu_seqlens, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                   ssm_state, conv_state, slot_idx=None, has_init=None, nthreads: int | None = None):
+    """Packed variable-length prefill on state slots. Sequence i owns packed rows
+    cu_seqlens[i] .. cu_seqlens[i+1]-1 of x, z, B, C, dt ([T, width]); it is an independent
+    prefill that starts from the states of its slot (or from zeros where has_init[i] == 0)
+    and leaves its final states in that slot (several sequences in one engine batch, each on
+    its own slot: gllm PR #86, section "Validation"). ``d.batch`` and ``d.seqlen`` are not
+    used. Returns y [T, H*P] and NEW state arrays; inputs are not modified."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    nseq = len(cu) - 1
+    slots = np.arange(nseq) if slot_idx is None else np.asarray(slot_idx)
+    init = np.ones(nseq, dtype=bool) if has_init is None else np.asarray(has_init) != 0
+    ssm_state = np.array(ssm_state, dtype=np.float64, copy=True)
+    conv_state = np.array(conv_state, dtype=np.float64, copy=True)
+    x, z, B, C, dt = (np.asarray(a) for a in (x, z, B, C, dt))
+    y = np.zeros((x.shape[0], d.nheads * d.headdim))
+    for i in range(nseq):
+        s0, s1 = int(cu[i]), int(cu[i + 1])
+        di = Dims(1, s1 - s0, d.nheads, d.headdim, d.ngroups, d.dstate, d.dconv, d.eps)
+        k = slots[i]
+        out = prefill(di, x[None, s0:s1], z[None, s0:s1], B[None, s0:s1], C[None, s0:s1], dt[None, s0:s1],
+                      A, D, conv_w, conv_b, dt_bias, norm_w,
+                      ssm_state[k][None] if init[i] else None, conv_state[k][None] if init[i] else None,
+                      nthreads=nthreads)
+        y[s0:s1] = out["y"][0]
+        ssm_state[k] = out["final_ssm"][0]
+        conv_state[k] = out["final_conv"][0]
+    return y, ssm_state, conv_state
+
+
 def decode_step(d: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
                 ssm_state, conv_state, slot_idx=None, nthreads: int | None = None):
     """One single-token decode step on state slots (returns y [b, H*P] and NEW state

@@ -104,3 +104,28 @@ def test_workspace_size_grows_with_tokens(lib):
     a = lib.ssd_mixer_prefill_workspace_size(ctypes.byref(_dims(seqlen=64).c()))
     b = lib.ssd_mixer_prefill_workspace_size(ctypes.byref(_dims(seqlen=640).c()))
     assert b > 5 * a
+
+
+def call_varlen(lib, d, cu=FAKE, ws_bytes=1 << 30, ssm=FAKE):
+    cd = d.c()
+    HP, GN = d.d_inner, d.ngroups * d.dstate
+    return lib.ssd_mixer_prefill_varlen(ctypes.byref(cd), cu, None, None, FAKE, HP, FAKE, HP, FAKE, GN, FAKE, GN,
+                                        FAKE, d.nheads, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ssm, FAKE,
+                                        FAKE, HP, FAKE, ws_bytes, None)
+
+
+def test_varlen_runs_the_tensor_core_shapes_only(lib):
+    tc = _dims(batch=3, seqlen=500, nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128)
+    assert lib.ssd_mixer_prefill_varlen_workspace_size(ctypes.byref(tc.c())) >= 256
+    for bad in (dict(act="f32"), dict(headdim=32), dict(nheads=6, ngroups=2)):
+        d = _dims(**{**dict(batch=3, seqlen=500, nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128), **bad})
+        assert lib.ssd_mixer_prefill_varlen_workspace_size(ctypes.byref(d.c())) == 0
+        assert call_varlen(lib, d) == sm.SSD_ERR_UNSUPPORTED
+
+
+def test_varlen_rejects_missing_pointers_and_small_workspace(lib):
+    d = _dims(batch=3, seqlen=500, nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128)
+    assert call_varlen(lib, d, cu=None) == sm.SSD_ERR_INVALID_ARG
+    assert call_varlen(lib, d, ssm=None) == sm.SSD_ERR_INVALID_ARG
+    assert call_varlen(lib, d, ws_bytes=16) == sm.SSD_ERR_INVALID_ARG
+    assert call_varlen(lib, d, cu=FAKE + 2) == sm.SSD_ERR_UNSUPPORTED   # cu_seqlens not 4-byte aligned

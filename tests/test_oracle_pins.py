@@ -369,3 +369,46 @@ def test_prefill_equals_prefill_then_decode_steps():
         assert rel(y, full["y"][:, t]) <= 1e-12
     assert rel(ssm[perm], full["final_ssm"]) <= 1e-12
     np.testing.assert_array_equal(conv[perm], full["final_conv"])
+
+
+def test_varlen_equal_lengths_equals_batched_prefill():
+    """Packed sequences of one length on identity slots, all continuing from their slots,
+    are the batched prefill row by row (bit for bit: the same per-row computation)."""
+    rng = np.random.default_rng(41)
+    d, inp = rand_problem(rng, b=3, L=17)
+    ref = oracle.prefill_dict(d, inp)
+    T = d.batch * d.seqlen
+    pk = {k: inp[k].reshape(T, -1) for k in ("x", "z", "B", "C", "dt")}
+    cu = np.arange(0, T + 1, d.seqlen)
+    y, ssm, conv = oracle.prefill_varlen(d, cu, pk["x"], pk["z"], pk["B"], pk["C"], pk["dt"], inp["A"], inp["D"],
+                                         inp["conv_w"], inp["conv_b"], inp["dt_bias"], inp["norm_w"],
+                                         inp["init_ssm"], inp["init_conv"])
+    assert np.array_equal(y, ref["y"].reshape(T, -1))
+    assert np.array_equal(ssm, ref["final_ssm"]) and np.array_equal(conv, ref["final_conv"])
+
+
+def test_varlen_slots_fresh_starts_and_empty_sequences():
+    """Slot mapping: a sequence with has_init = 0 equals a prefill from zero states; an empty
+    sequence leaves its slot's states as they were; untouched slots are unchanged."""
+    rng = np.random.default_rng(42)
+    d, inp = rand_problem(rng, b=1, L=30, init=False)
+    H, P, N, Cc = d.nheads, d.headdim, d.dstate, d.xbc_channels
+    nslots = 5
+    ssm0 = 0.1 * rng.standard_normal((nslots, H, P, N))
+    conv0 = rng.standard_normal((nslots, Cc, 3))
+    lens = [12, 0, 18]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    pk = {k: inp[k][0] for k in ("x", "z", "B", "C", "dt")}
+    slots, has_init = [3, 1, 0], [0, 1, 1]
+    y, ssm, conv = oracle.prefill_varlen(d, cu, pk["x"], pk["z"], pk["B"], pk["C"], pk["dt"], inp["A"], inp["D"],
+                                         inp["conv_w"], inp["conv_b"], inp["dt_bias"], inp["norm_w"],
+                                         ssm0, conv0, slot_idx=slots, has_init=has_init)
+    par = {k: inp[k] for k in ("A", "D", "conv_w", "conv_b", "dt_bias", "norm_w")}
+    fresh = oracle.prefill(Dims(1, 12, H, P, d.ngroups, N, 4, d.eps), *(inp[k][:, :12] for k in ("x", "z", "B", "C", "dt")),
+                           *par.values())
+    assert np.array_equal(y[:12], fresh["y"][0]) and np.array_equal(ssm[3], fresh["final_ssm"][0])
+    cont = oracle.prefill(Dims(1, 18, H, P, d.ngroups, N, 4, d.eps), *(inp[k][:, 12:30] for k in ("x", "z", "B", "C", "dt")),
+                          *par.values(), ssm0[0][None], conv0[0][None])
+    assert np.array_equal(y[12:30], cont["y"][0]) and np.array_equal(conv[0], cont["final_conv"][0])
+    for k in (1, 2, 4):     # the empty sequence's slot and the untouched slots
+        assert np.array_equal(ssm[k], ssm0[k]) and np.array_equal(conv[k], conv0[k])
