@@ -146,8 +146,80 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.ssp = (float*)(ws + wl.ssp);
     p.bc_conv = ws + wl.bc_conv;
     cudaStream_t st = (cudaStream_t)stream;
+
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
     if ((tc ? ssd::launch_prefill_ws(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+size_t ssd_mixer_prefill_state_workspace_size(const ssd_dims* d)
+{
+    if (check_dims(d, false) != SSD_OK ||
+        !ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups))
+        return 0;
+    return ssd::prefill_workspace_layout(d->batch, d->seqlen, d->batch * d->seqlen, d->nheads, d->headdim,
+                                         d->ngroups, d->dstate, d->chunk, d->act)
+        .total;
+}
+
+ssd_status ssd_mixer_prefill_state(const ssd_dims* d, const void* x, int64_t x_ld, const void* B, int64_t B_ld,
+                                   const void* C, int64_t C_ld, const void* dt, int64_t dt_ld, const float* A,
+                                   const float* conv_w, const float* conv_b, const float* dt_bias,
+                                   const float* init_ssm_state, const void* init_conv_state,
+                                   float* final_ssm_state, void* final_conv_state, float* decay,
+                                   void* workspace, size_t workspace_bytes, void* stream)
+{
+    const ssd_status ds = check_dims(d, false);
+    if (ds != SSD_OK) return ds;
+    if (!ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups))
+        return SSD_ERR_UNSUPPORTED;
+    const size_t es = 2;
+    const int64_t HP = (int64_t)d->nheads * d->headdim, GN = (int64_t)d->ngroups * d->dstate;
+    if (!A || !conv_w || !conv_b || !dt_bias || !final_ssm_state || !final_conv_state) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(conv_w) || !aligned16(final_ssm_state) || (init_ssm_state && !aligned16(init_ssm_state)) ||
+        (init_conv_state && ((uintptr_t)init_conv_state % es)) || ((uintptr_t)final_conv_state % es) ||
+        (decay && ((uintptr_t)decay & 3u)))
+        return SSD_ERR_UNSUPPORTED;
+    const ssd::WorkspaceLayout wl = ssd::prefill_workspace_layout(d->batch, d->seqlen, d->batch * d->seqlen, d->nheads,
+                                                                  d->headdim, d->ngroups, d->dstate, d->chunk, d->act);
+    if (!workspace || workspace_bytes < wl.total || ((uintptr_t)workspace & 255u)) return SSD_ERR_INVALID_ARG;
+    if (d->seqlen > 0 && d->batch > 0) {
+        if (!x || !B || !C || !dt) return SSD_ERR_INVALID_ARG;
+        if (!row_ok(x, x_ld, HP, es, true) || !row_ok(B, B_ld, GN, es, true) || !row_ok(C, C_ld, GN, es, true) ||
+            !row_ok(dt, dt_ld, d->nheads, es, false))
+            return SSD_ERR_UNSUPPORTED;
+    }
+    ssd::PrefillParams p{};
+    p.b = d->batch; p.L = d->seqlen;
+    p.H = d->nheads; p.P = d->headdim; p.G = d->ngroups; p.N = d->dstate; p.K = d->dconv;
+    p.Q = d->chunk; p.eps = d->eps; p.act = d->act;
+    p.nc = (p.L + p.Q - 1) / p.Q;
+    p.x = x; p.B = B; p.C = C; p.dt = dt;
+    p.x_ld = x_ld; p.B_ld = B_ld; p.C_ld = C_ld; p.dt_ld = dt_ld;
+    p.A = A; p.conv_w = conv_w; p.conv_b = conv_b; p.dt_bias = dt_bias;
+    p.init_ssm = init_ssm_state; p.init_conv = init_conv_state;
+    p.final_ssm = final_ssm_state; p.final_conv = final_conv_state; p.decay = decay;
+    char* ws = (char*)workspace;
+    p.status = (int*)(ws + wl.status);
+    p.ssp = (float*)(ws + wl.ssp);
+    p.bc_conv = ws + wl.bc_conv;
+    if (ssd::launch_prefill_state_ws(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+ssd_status ssd_mixer_state_pass(int64_t batch, int32_t nheads, int32_t headdim, int32_t dstate, int32_t r,
+                                const float* decay, const float* state, const float* init, float* out,
+                                void* stream)
+{
+    if (batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || r < 0) return SSD_ERR_INVALID_ARG;
+    if (((int64_t)headdim * dstate) % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (!out || (r > 0 && (!decay || !state))) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(out) || (state && !aligned16(state)) || (init && !aligned16(init)) ||
+        (decay && ((uintptr_t)decay & 3u)))
+        return SSD_ERR_UNSUPPORTED;
+    if (ssd::launch_state_pass(batch, nheads, headdim, dstate, r, decay, state, init, out, (cudaStream_t)stream) !=
+        cudaSuccess)
         return SSD_ERR_CUDA;
     return SSD_OK;
 }

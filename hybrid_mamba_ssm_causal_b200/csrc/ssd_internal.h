@@ -46,6 +46,8 @@ struct PrefillParams {
     const int32_t* cu_seqlens;
     const int32_t* slot_idx;
     const uint8_t* has_init;
+    // state-only pass (ssd_mixer_prefill_state): exp(sum_t delta_t * A) per (row, head), [b][H]
+    float* decay;
 
     SSD_HD int64_t HP() const { return (int64_t)H * P; }
     SSD_HD int64_t GN() const { return (int64_t)G * N; }
@@ -86,8 +88,14 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int
 // one cluster (prefill_tc_split).
 bool prefill_tc_supported(int act, int P, int N, int H, int G);
 bool prefill_tc_split(int H, int G);
+// The state-only pass on the tensor-core path: final states and decay, no output rows.
+cudaError_t launch_prefill_state_ws(const PrefillParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream);
 int prefill_ws_partials_per_head();
+
+// H_in(r) of a sequence split into pieces: init (NULL = zeros) carried through pieces 0..r-1.
+cudaError_t launch_state_pass(int64_t b, int H, int P, int N, int r, const float* decay, const float* state,
+                              const float* init, float* out, cudaStream_t stream);
 
 bool prefill_simt_supported(int P, int N);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t stream);

@@ -145,7 +145,9 @@ struct WsMaps {
     CUtensorMap x, B, C, z, y;
 };
 
-template <int R, bool SPLIT>
+// STATE_ONLY: the state-only pass (final states and decay of a prefill, no output rows): the
+// conv of x and B, B'^T(x'w) and the state recurrence; C's raw rows only for the conv state.
+template <int R, bool SPLIT, bool STATE_ONLY>
 __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillParams p, const __grid_constant__ WsMaps maps)
 {
     using Lo = WsLayout<R>;
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         cw[0] = w.x; cw[2] = w.y; cw[4] = w.z; cw[6] = w.w;
         s_cb[c] = p.conv_b[ch];
     }
-    if (tid < kP) s_nw[tid] = p.norm_w[(int64_t)h * kP + tid];
+    if (!STATE_ONLY && tid < kP) s_nw[tid] = p.norm_w[(int64_t)h * kP + tid];
     if (tid == 0) {
         mbar_init(bar0, 1);
         mbar_init(bar1, 1);
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const float A2 = p.A[h] * 1.4426950408889634f;
-    const float Dh = p.D[h];
+    const float Dh = STATE_ONLY ? 0.0f : p.D[h];
     const float bias = p.dt_bias[h];
     bool ok = true;
 
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     !mbar_wait_cluster(barF2 + 8 * (uint32_t)((k - 1) & 1), (uint32_t)(((k - 1) >> 1) & 1), kWaitLimit))
                     ok = false;
                 if (k >= 2 && ok && !mbar_wait_bounded(barE2 + 8 * sl, (uint32_t)(((k - 2) >> 1) & 1), kWaitLimit)) ok = false;
-                mbar_arrive_expect_tx(barX, (uint32_t)(R - 1) * 2 * kSliceBytes);
+                mbar_arrive_expect_tx(barX, (uint32_t)(R - 1) * (STATE_ONLY ? 1 : 2) * kSliceBytes);
             }
             // this block's raw B/C rows (its x rows may still be in flight)
             if (ok && !mbar_wait_bounded(barTB, (uint32_t)(k & 1), kWaitLimit)) ok = false;
@@ -422,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 }
             };
             // this CTA's slice of B' and C' first, so its copies to the peers overlap the x' conv
-            conv_vectors(std::integral_constant<int, kVX>{}, std::integral_constant<int, kVBC>{});
+            conv_vectors(std::integral_constant<int, kVX>{}, std::integral_constant<int, STATE_ONLY ? NS / 8 : kVBC>{});
             fence_async_smem();
             named_sync(kBarProd, kProd);
             // one duty per warp (lane 0), so that none lags the x' conv by more than one TMA or
@@ -431,10 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             if ((tid & 31) == 0) {
                 if (warp == 1) {
                     if (k + 1 < nblk) load_bc(k + 1);
-                } else if (warp >= 2 && warp - 2 < 2 * (R - 1)) {
-                    const int idx = warp - 2;
-                    const uint32_t rr = (uint32_t)((q + 1 + idx / 2) % R);
-                    const uint32_t src = (idx & 1 ? aC : aB) + slice_off;
+                } else if (warp >= 2 && warp - 2 < (STATE_ONLY ? 1 : 2) * (R - 1)) {
+                    const int idx = warp - 2, nm = STATE_ONLY ? 1 : 2;   // matrices sent (B, or B and C)
+                    const uint32_t rr = (uint32_t)((q + 1 + idx / nm) % R);
+                    const uint32_t src = (idx % nm ? aC : aB) + slice_off;
                     bulk_copy_to_peer(cluster_map(src, rr), src, kSliceBytes, cluster_map(barX, rr));
                 }
             }
@@ -453,12 +455,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 const uint32_t id_ys = idesc_bf16(128, 64, 0, 1);
                 const uint32_t id_s = idesc_bf16(128, 64, 1, 1);
                 const uint32_t colYs = kColYs0 + 64 * (uint32_t)sl;
+                if constexpr (!STATE_ONLY) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tmem + kColCB, sdesc(aC + kk * 4096, 2048, 128), sdesc(aB + kk * 4096, 2048, 128), id_cb, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tmem + kColCB, sdesc(aC + kk * 4096, 2048, 128), sdesc(aB + kk * 4096, 2048, 128), id_cb, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tmem + colYs, sdesc(aC + kk * 4096, 2048, 128), sdesc(aH + kk * 2048, 1024, 128), id_ys, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tmem + colYs, sdesc(aC + kk * 4096, 2048, 128), sdesc(aH + kk * 2048, 1024, 128), id_ys, kk > 0);
+                }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16(tmem + kColS, sdesc(aB + kk * 256, 128, 2048), sdesc(aXW + kk * 2048, 1024, 128), id_s, kk > 0);
@@ -499,6 +503,39 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 ((__nv_bfloat16*)p.final_conv)[(sidx * Cc + staged_channel(c)) * 3 + kk] = v;
             }
         }
+    } else if constexpr (STATE_ONLY) {
+        // ================= consumer of the state-only pass (warps 8..15) =================
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        float lam_tot = 0.0f;   // sum of delta*A over the row, log2 units
+        for (int64_t k = 0; k < nblk; ++k) {
+            const int sl = (int)(k & 1);
+            const uint32_t par = (uint32_t)(k & 1);
+            if (ok && !mbar_wait_bounded(barP, par, kWaitLimit)) ok = false;
+            if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
+            fence_after_sync();
+            const float lam_end = s_lam[sl * kT + kT - 1];
+            lam_tot += lam_end;
+            float s_[32];
+            tmem_ld32(tmem + lane_base + kColS + chalf * 32, s_);
+            tmem_wait_ld();
+            const float2 aend = splat2(ex2(lam_end));
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float2 hv = fma2(aend, make_float2(H[i], H[i + 1]), make_float2(s_[i], s_[i + 1]));
+                H[i] = hv.x;
+                H[i + 1] = hv.y;
+            }
+            fence_before_sync();
+            named_sync(kBarCons, kThreads - kProd);
+            if (tid == kProd) {
+                mbar_arrive_local(barC);             // S^T read: the next block's MMA may overwrite it
+                mbar_arrive_local(barE2 + 8 * sl);   // the cumsum slot is free
+            }
+        }
+        float* fs = p.final_ssm + (sidx * p.H + h) * (int64_t)kP * kN;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) fs[(int64_t)(chalf * 32 + i) * kN + crow] = H[i];
+        if (tid == kProd && p.decay) p.decay[bi * p.H + h] = ex2(lam_tot);
     } else {
         // =========================== consumer (warps 8..15) ===========================
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -811,7 +848,7 @@ __global__ void __launch_bounds__(256) ws_bc_conv_out_kernel(PrefillParams p)
     ((__nv_bfloat16*)p.final_conv)[(sidx * p.Cc() + p.HP()) * 3 + r] = ((const __nv_bfloat16*)p.bc_conv)[e];
 }
 
-template <int R, bool SPLIT>
+template <int R, bool SPLIT, bool STATE_ONLY = false>
 cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
 {
     using Lo = WsLayout<R>;
@@ -822,11 +859,13 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     if (p.L > 0) {   // no block, no load: the maps stay unused
         if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, mL, mb, kP / 8) ||
             !encode_rows(&maps.B, p.B, p.GN(), p.B_ld, mL, mb, Lo::NS / 8) ||
-            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, mL, mb, Lo::NS / 8) ||
-            !encode_tile(&maps.z, p.z, p.HP(), p.z_ld, mL, mb) || !encode_tile(&maps.y, p.y, p.HP(), p.y_ld, mL, mb))
+            !encode_rows(&maps.C, p.C, p.GN(), p.C_ld, mL, mb, Lo::NS / 8))
+            return cudaErrorInvalidValue;
+        if (!STATE_ONLY &&
+            (!encode_tile(&maps.z, p.z, p.HP(), p.z_ld, mL, mb) || !encode_tile(&maps.y, p.y, p.HP(), p.y_ld, mL, mb)))
             return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT, STATE_ONLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::TOTAL);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -842,11 +881,11 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     {
-        LaunchScope ls("tc_prefill", st);
-        e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT>, p, maps);
+        LaunchScope ls(STATE_ONLY ? "tc_prefill_state" : "tc_prefill", st);
+        e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT, STATE_ONLY>, p, maps);
         if (e != cudaSuccess) return e;
     }
-    if (SPLIT && p.rows() > 0) {
+    if (SPLIT && !STATE_ONLY && p.rows() > 0) {
         LaunchScope ls("tc_norm_finish", st);
         const int64_t warps = p.rows() * p.G;
         ws_norm_finish_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
@@ -866,6 +905,16 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
 
 // Groups of 2 or 4 heads: one cluster per group (fused norm); wider groups: clusters of 4
 // heads and the norm finished by ws_norm_finish_kernel.
+cudaError_t launch_prefill_state_ws(const PrefillParams& p, cudaStream_t stream)
+{
+    if (p.b == 0) return cudaSuccess;
+    switch (p.H / p.G) {
+    case 2: return launch_ws<2, false, true>(p, stream);
+    case 4: return launch_ws<4, false, true>(p, stream);
+    }
+    return launch_ws<4, true, true>(p, stream);
+}
+
 cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream)
 {
     if (p.b == 0) return cudaSuccess;
@@ -885,5 +934,7 @@ bool prefill_tc_supported(int act, int P, int N, int H, int G)
 }
 
 bool prefill_tc_split(int H, int G) { return H / G > 4; }
+
+
 
 }  // namespace ssd

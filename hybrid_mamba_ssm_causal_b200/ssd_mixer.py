@@ -32,7 +32,8 @@ SSD_F32, SSD_BF16 = 0, 1
 SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_decode_step",
            "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version",
            "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read",
-           "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen")
+           "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
+           "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass")
 
 
 class SsdError(RuntimeError):
@@ -111,6 +112,14 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_prefill_varlen.argtypes = ([ctypes.POINTER(_CDims), P, P, P] + [P, I64] * 5 + [FP] * 6 +
                                              [FP, P, P, I64, P, ctypes.c_size_t, V])
     lib.ssd_mixer_prefill_varlen.restype = ctypes.c_int
+    lib.ssd_mixer_prefill_state_workspace_size.argtypes = [ctypes.POINTER(_CDims)]
+    lib.ssd_mixer_prefill_state_workspace_size.restype = ctypes.c_size_t
+    lib.ssd_mixer_prefill_state.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 4 + [FP] * 4 +
+                                            [FP, P, FP, P, FP, P, ctypes.c_size_t, V])
+    lib.ssd_mixer_prefill_state.restype = ctypes.c_int
+    lib.ssd_mixer_state_pass.argtypes = [I64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                         FP, FP, FP, FP, V]
+    lib.ssd_mixer_state_pass.restype = ctypes.c_int
     lib.ssd_mixer_workspace_status.argtypes = [P, V]
     lib.ssd_mixer_workspace_status.restype = ctypes.c_int
     lib.ssd_status_string.argtypes = [ctypes.c_int]
@@ -242,6 +251,39 @@ def ssd_mixer_prefill_varlen(dims: Dims, cu_seqlens, slot_idx, has_init, x, z, B
         _dev(conv_state, "conv_state"), py, y_ld, _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "ssd_mixer_prefill_varlen")
+
+
+def ssd_mixer_prefill_state_workspace_size(dims: Dims) -> int:
+    cd = dims.c()
+    return int(load_library().ssd_mixer_prefill_state_workspace_size(ctypes.byref(cd)))
+
+
+def ssd_mixer_prefill_state(dims: Dims, x, B, C, dt, A, conv_w, conv_b, dt_bias, init_ssm_state,
+                            init_conv_state, final_ssm_state, final_conv_state, decay, workspace,
+                            stream=None) -> None:
+    """State-only prefill: final states and the per-(row, head) decay, no output rows."""
+    lib = load_library()
+    rows = dims.batch * dims.seqlen
+    GN = dims.ngroups * dims.dstate
+    args = []
+    for t, name, w in ((x, "x", dims.d_inner), (B, "B", GN), (C, "C", GN), (dt, "dt", dims.nheads)):
+        args += list(_rows(t, name, rows, w))
+    cd = dims.c()
+    st = lib.ssd_mixer_prefill_state(
+        ctypes.byref(cd), *args, _dev(A, "A"), _dev(conv_w, "conv_w"), _dev(conv_b, "conv_b"),
+        _dev(dt_bias, "dt_bias"), _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
+        _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"), _dev(decay, "decay"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "ssd_mixer_prefill_state")
+
+
+def ssd_mixer_state_pass(r: int, decay, state, init, out, stream=None) -> None:
+    """State entering piece r of a split sequence: decay [npieces, b, H], state
+    [npieces, b, H, P, N] (zero-start final states of the pieces), init [b, H, P, N] or None."""
+    b, H, P, N = out.shape
+    st = load_library().ssd_mixer_state_pass(b, H, P, N, r, _dev(decay, "decay"), _dev(state, "state"),
+                                             _dev(init, "init"), _dev(out, "out"), _stream(stream))
+    _check(st, "ssd_mixer_state_pass")
 
 
 def ssd_mixer_decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,

@@ -126,6 +126,48 @@ SSD_API ssd_status ssd_mixer_prefill(const ssd_dims* dims,
                              void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* Bytes of device workspace ssd_mixer_prefill_state needs for `dims`; 0 when the dims are
+ * invalid or the shape is one the state-only pass does not run. */
+SSD_API size_t ssd_mixer_prefill_state_workspace_size(const ssd_dims* dims);
+
+/* State-only prefill: the final states of ssd_mixer_prefill, without the output rows, plus
+ * the decay of each row's whole piece. A piece of a long sequence then hands its state to the
+ * next piece without computing its own outputs first, which is the state passing that a
+ * sequence split across devices needs (Modalities PR #459, section "Next steps for
+ * production at scale", item "MTP and long-context": the long-context phase wants context
+ * parallelism with Mamba state passing; section "Testing": state passing across a split
+ * sequence). With S_r the final state of piece r computed from a zero initial state and a_r
+ * its decay, the state entering piece r+1 is a_r * (state entering piece r) + S_r.
+ *
+ * Same inputs and state layouts as ssd_mixer_prefill, without z, D and norm_w (C is read
+ * only for its final conv state). Outputs: final_ssm_state, final_conv_state, and decay
+ * [b][H] fp32 (NULL = not wanted): exp(A[h] * sum over the row's tokens of delta_t[h]).
+ * Runs the tensor-core kernel only (bf16, P = 64, N = 128, 2 or a multiple of 4 heads per
+ * group); other shapes return SSD_ERR_UNSUPPORTED. Final states may alias initial ones. */
+SSD_API ssd_status ssd_mixer_prefill_state(const ssd_dims* dims,
+                                   const void* x, int64_t x_ld,
+                                   const void* B, int64_t B_ld,
+                                   const void* C, int64_t C_ld,
+                                   const void* dt, int64_t dt_ld,
+                                   const float* A, const float* conv_w, const float* conv_b,
+                                   const float* dt_bias,
+                                   const float* init_ssm_state, const void* init_conv_state,
+                                   float* final_ssm_state, void* final_conv_state,
+                                   float* decay,
+                                   void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/* State passing between the pieces of a split sequence (the companion of
+ * ssd_mixer_prefill_state; same citations): writes the state entering piece r,
+ *   H_in(0) = init,  H_in(j+1) = decay[j] * H_in(j) + state[j],  j < r,
+ * where state[j] is piece j's final SSM state from a zero initial state and decay[j] its
+ * decay. decay [npieces][batch][nheads] fp32; state [npieces][batch][nheads][headdim][dstate]
+ * fp32 (only pieces 0..r-1 are read); init [batch][nheads][headdim][dstate] or NULL = zeros;
+ * out the same shape (may alias init). Device pointers, 16-byte aligned (decay: 4). */
+SSD_API ssd_status ssd_mixer_state_pass(int64_t batch, int32_t nheads, int32_t headdim, int32_t dstate,
+                                int32_t r, const float* decay, const float* state,
+                                const float* init, float* out, void* stream);
+
 /* Bytes of device workspace ssd_mixer_prefill_varlen needs for `dims` (dims->batch
  * sequences, dims->seqlen packed tokens in total); 0 when the dims are invalid or the
  * shape is one the packed entry point does not run. */

@@ -194,6 +194,16 @@ def prefill_dict(d: Dims, inp: dict, **kw):
                    inp.get("init_ssm"), inp.get("init_conv"), **kw)
 
 
+def decay(dt, A, dt_bias):
+    """exp(A[h] * sum_t delta_t[h]) per (row, head), delta = softplus(dt + dt_bias): the product
+    of the per-token factors exp(delta_t A) of the state recurrence, i.e. the factor by which
+    a prefill over these tokens carries its initial SSM state into its final one.
+    dt [b, L, H]; returns [b, H]."""
+    u = np.asarray(dt, np.float64) + np.asarray(dt_bias, np.float64)
+    delta = np.where(u > 20.0, u, np.log1p(np.exp(np.minimum(u, 20.0))))
+    return np.exp(np.asarray(A, np.float64) * delta.sum(axis=1))
+
+
 def prefill_varlen(d: Dims, cu_seqlens, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
                    ssm_state, conv_state, slot_idx=None, has_init=None, nthreads: int | None = None):
     """Packed variable-length prefill on state slots. Sequence i owns packed rows

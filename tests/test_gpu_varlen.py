@@ -76,11 +76,13 @@ def test_varlen_all_sequences_empty():
     run_varlen(8, 2, lens=[0, 0, 0], slots=[2, 0, 1], has_init=[1, 0, 1], nslots=4, seed=54)
 
 
-def test_wide_groups_final_states_may_alias_initial_states():
+@pytest.mark.parametrize("b,L", [(2, 333), (1, 600)])
+def test_wide_groups_final_states_may_alias_initial_states(b, L):
     """Plain prefill, bf16, 8 heads per group (two clusters of 4 per group), with the final
-    states written over the initial ones."""
+    states written over the initial ones (the second shape would otherwise be cut into two
+    segments)."""
     base = WORKLOADS["small_bf16"]
-    w = base.with_(batch=2, seqlen=333, nheads=16, headdim=64, ngroups=2, dstate=128, chunk=128,
+    w = base.with_(batch=b, seqlen=L, nheads=16, headdim=64, ngroups=2, dstate=128, chunk=128,
                    init_ssm_std=0.1, init_conv_std=1.0, seed=55)
     inp = make_prefill_inputs(w)
     d = dims_of(w)

@@ -412,3 +412,27 @@ def test_varlen_slots_fresh_starts_and_empty_sequences():
     assert np.array_equal(y[12:30], cont["y"][0]) and np.array_equal(conv[0], cont["final_conv"][0])
     for k in (1, 2, 4):     # the empty sequence's slot and the untouched slots
         assert np.array_equal(ssm[k], ssm0[k]) and np.array_equal(conv[k], conv0[k])
+
+
+def test_final_state_is_linear_in_the_initial_state_with_the_decay_factor():
+    """final(H0) = decay * H0 + final(0) for one piece (the recurrence is linear in the state,
+    and the product of its per-token factors exp(delta_t A) is the decay); the basis of
+    passing the state between the pieces of a split sequence."""
+    rng = np.random.default_rng(43)
+    d, inp = rand_problem(rng, b=2, L=37, init=True)
+    with_init = oracle.prefill_dict(d, inp)
+    zero = oracle.prefill_dict(d, dict(inp, init_ssm=None))
+    a = oracle.decay(inp["dt"], inp["A"], inp["dt_bias"])
+    pred = a[:, :, None, None] * inp["init_ssm"] + zero["final_ssm"]
+    assert np.max(np.abs(pred - with_init["final_ssm"])) <= 1e-12 * np.max(np.abs(with_init["final_ssm"]))
+    # and pieces chain: two pieces folded equal one prefill over both
+    d1 = Dims(d.batch, 20, d.nheads, d.headdim, d.ngroups, d.dstate, d.dconv, d.eps)
+    d2 = Dims(d.batch, 17, d.nheads, d.headdim, d.ngroups, d.dstate, d.dconv, d.eps)
+    cut = lambda v, s: v[:, s] if v is not None and v.ndim == 3 and v.shape[1] == d.seqlen else v
+    p1 = {k: cut(v, slice(0, 20)) for k, v in inp.items()}
+    p2 = {k: cut(v, slice(20, 37)) for k, v in inp.items()}
+    r1 = oracle.prefill_dict(d1, p1)
+    r2z = oracle.prefill_dict(d2, dict(p2, init_ssm=None, init_conv=r1["final_conv"]))
+    a2 = oracle.decay(p2["dt"], inp["A"], inp["dt_bias"])
+    chained = a2[:, :, None, None] * r1["final_ssm"] + r2z["final_ssm"]
+    assert np.max(np.abs(chained - with_init["final_ssm"])) <= 1e-12 * np.max(np.abs(with_init["final_ssm"]))
