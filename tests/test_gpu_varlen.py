@@ -96,3 +96,43 @@ def test_wide_groups_final_states_may_alias_initial_states(b, L):
     assert_close("y", y, ref["y"], tol)
     assert_close("final_ssm (aliased)", ssm, ref["final_ssm"], tol)
     assert_close("final_conv (aliased)", conv, ref["final_conv"], tol)
+
+
+def test_one_token_sequences_match_the_decode_step():
+    """Mixed prefill and decode in one packed call: one-token sequences give the same outputs
+    and slot states as ssd_mixer_decode_step on the same slots (both run the recurrence once
+    from the slot's states), next to a longer prefill on another slot."""
+    H, G, nslots = 8, 2, 6
+    lens = [1, 200, 1, 1]
+    slots = [4, 1, 0, 5]
+    T = sum(lens)
+    w = WORKLOADS["small_bf16"].with_(batch=1, seqlen=T, nheads=H, headdim=64, ngroups=G, dstate=128,
+                                      chunk=128, init_ssm_std=0.0, init_conv_std=0.0, seed=57)
+    inp = make_prefill_inputs(w)
+    rng = np.random.default_rng(58)
+    ssm0 = torch.from_numpy((0.1 * rng.standard_normal((nslots, H, 64, 128))).astype(np.float32)).cuda()
+    conv0 = torch.from_numpy(round_bf16(rng.standard_normal((nslots, w.xbc_channels, 3))).astype(np.float32))
+    conv0 = conv0.to(torch.bfloat16).cuda()
+    dv = to_dev({k: np.ascontiguousarray(inp[k][0]) for k in SEQ}, "bf16")
+    par = to_dev({k: inp[k] for k in PARAMS}, "bf16")
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    # packed call
+    ssm_a, conv_a = ssm0.clone(), conv0.clone()
+    y_a = torch.empty(T, H * 64, dtype=torch.bfloat16, device="cuda")
+    d = sm.Dims(len(lens), T, H, 64, G, 128, 128, 4, w.eps, "bf16")
+    ws = torch.empty(sm.ssd_mixer_prefill_varlen_workspace_size(d), dtype=torch.uint8, device="cuda")
+    sm.ssd_mixer_prefill_varlen(d, cu, torch.tensor(slots, dtype=torch.int32, device="cuda"), None,
+                                *(dv[k] for k in SEQ), *(par[k] for k in PARAMS), ssm_a, conv_a, y_a, ws)
+    # decode steps for the one-token sequences
+    ones = [i for i, n in enumerate(lens) if n == 1]
+    rows = [int(cu[i]) for i in ones]
+    ssm_b, conv_b = ssm0.clone(), conv0.clone()
+    dd = sm.Dims(len(ones), 1, H, 64, G, 128, 1, 4, w.eps, "bf16")
+    y_b = sm.decode_step(dd, *(dv[k][rows].contiguous() for k in SEQ), *(par[k] for k in PARAMS), ssm_b, conv_b,
+                         torch.tensor([slots[i] for i in ones], dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    for j, i in enumerate(ones):
+        assert_close(f"y of one-token sequence {i}", y_a[rows[j]], y_b[j].float().cpu().numpy(), TOL["bf16"])
+        k = slots[i]
+        assert_close(f"ssm slot {k}", ssm_a[k], ssm_b[k].cpu().numpy(), TOL["bf16"])
+        assert torch.equal(conv_a[k], conv_b[k]), f"conv slot {k}"
