@@ -267,6 +267,25 @@ def workload_desc(w):
             f"conv{w.dconv} Q{w.chunk} {w.act}, then 1 decode step")
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, units_per_rank_step: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the units every rank processed per step over the step time (weak
+    scaling: each rank runs its own replica of the workload)."""
+    return world * units_per_rank_step / (ms_per_step * 1e-3)
+
+
 # ------------------------------------------------------------------ our arm
 
 def main():
@@ -295,12 +314,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     w = WORKLOADS[WORKLOAD]
     inp = make_prefill_inputs(w)
@@ -362,9 +377,9 @@ def main():
     lib.ssd_mixer_profile_enable(0)
     barrier()
     ms_local = e0.elapsed_time(e1) / a.steps
-    ms = max_over_ranks(ms_local)
+    ms = rank_max(ms_local)
     tok_step = w.batch * (w.seqlen + 1)
-    value = world * tok_step / (ms * 1e-3)
+    value = job_value(world, tok_step, ms)
 
     # dominant kernel and its roofline
     dom = max(per_kernel.items(), key=lambda kv: kv[1][0]) if per_kernel else None
@@ -409,8 +424,8 @@ def main():
             e2e_step(s)
         f1.record(stream)
         torch.cuda.synchronize()
-        ems = max_over_ranks(f0.elapsed_time(f1) / a.steps)
-        e2e = {"value": world * tok_step / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        ems = rank_max(f0.elapsed_time(f1) / a.steps)
+        e2e = {"value": job_value(world, tok_step, ems), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
     # decode workload: 256 sequences, 1000 single-token steps, state in place
@@ -443,12 +458,12 @@ def main():
             dstep(s)
         g1.record(stream)
         torch.cuda.synchronize()
-        dms = max_over_ranks(g0.elapsed_time(g1) / a.decode_steps)
+        dms = rank_max(g0.elapsed_time(g1) / a.decode_steps)
         db = decode_bytes(wd, wd.batch)
         ach = db / (dms * 1e-3) / 1e9
         decode = {"workload": f"decode_bf16: b{wd.batch} H{wd.nheads}xP{wd.headdim} G{wd.ngroups} N{wd.dstate} "
                               f"fp32 state, {a.decode_steps} steps",
-                  "value": world / (dms * 1e-3), "unit": "steps/s", "tokens_per_s": world * wd.batch / (dms * 1e-3),
+                  "value": job_value(world, 1, dms), "unit": "steps/s", "tokens_per_s": job_value(world, wd.batch, dms),
                   "us_per_step": dms * 1e3,
                   "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                                "frac": ach / hbm, "traffic": measured_traffic("decode_step"),
