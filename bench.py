@@ -125,12 +125,38 @@ TRAFFIC_SUMMARIES = {"tc_prefill": "profiles/ssd_prefill_ws_small_bf16.md",
                      "decode_step": "profiles/decode_step_decode_bf16.md"}
 
 
+def code_only(text: str) -> str:
+    """C++/CUDA source without its comments and with whitespace collapsed: the part that
+    decides what the compiled kernel does."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                                   # string or char literal, kept whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def sources_sha256(name: str) -> str:
+    """Hash of the code (comments and layout ignored) of the files a kernel is built from."""
     import hashlib
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[name]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -9,20 +9,32 @@
 //   M_ij = CB_ij exp(lam_i - lam_j) delta_j (j <= i), Yi = M x',
 //   y = Yi + exp(lam_i) Ys + D x',  g = y SiLU(z),  out = g / rms_group(g) * norm_w,
 //   H <- exp(lam_end) H + S.
-// Each CTA owns one head of one batch row; the heads of a cluster share the B/C conv
-// (each CTA convolves a slice and bulk-copies it into every peer) and, when the cluster
-// holds the whole group, the norm's per-token sums of squares (DSMEM).
+// Each CTA owns one head of one sequence; the heads of a cluster share the B/C conv (each
+// CTA convolves a slice and bulk-copies it into every peer) and, when the cluster holds the
+// whole group, the norm's per-token sums of squares (st.async into every peer).
+//
+// Data movement: the raw x, B and C rows of a block (with the 3-token conv halo) arrive by
+// TMA, one box per kind of channel; z is read and y written through 128-byte-swizzled TMA
+// tiles; the decay-masked M goes from registers into TMEM and feeds M x' as the TMEM
+// A operand.
 //
 // Roles (512 threads):
-//   producer warps 0..7  : raw loads (cp.async), softplus + cumsum, conv + SiLU into the
-//                          operand tiles, the slice exchange, and (thread 0) the MMAs on
-//                          C'B'^T, C'H^T and B'^T(x'w) for block k;
+//   producer warps 0..7  : for block k, the conv + SiLU of this CTA's B'/C' slice, then one
+//                          duty per warp (warp 1 the TMA refill of the next raw B/C rows,
+//                          warps 2.. one slice copy each to a peer), the conv + SiLU of x' and
+//                          x'w, and (thread 0) the MMAs C'B'^T, C'H^T and B'^T(x'w) once the
+//                          peers' slices are in; warps 4..7 then the softplus + cumsum of
+//                          block k+1;
 //   consumer warps 8..15 : for block k-1 meanwhile: the masked decay product M, the state
-//                          update, (thread 256) the MMA M x', the epilogue and the norm.
+//                          update, (thread 256) the MMA M x', the epilogue, and the group
+//                          norm of block k-2.
+// Variants: packed variable-length sequences on state slots (a CTA reads its sequence's
+// rows, length and slot from device arrays), and STATE_ONLY (final states and decay only).
 // Hand-offs use mbarriers (all waits bounded):
 //   bar0   MMA1-3 of a block done (tensor-core commit)     bar1  MMA4 done
 //   barX   the peers' B'/C' slices of a block have landed (bulk-copy transaction bytes)
-//   barP   producer: softplus/cumsum and x' of a block are in shared memory
+//   barP   producer: this block's x', x'w and cumsum are in shared memory (arrived just
+//          before MMA1-3 are issued)
 //   barC   consumer: C'B'^T and S^T read from TMEM, H^T of the next block written
 //   barE2  consumer: a block's x' and cumsum buffers are free again (2 slots by parity)
 //   barF2  every CTA of the cluster: its MMA1-3 of a block are done (2 slots; one arrival per
@@ -31,6 +43,7 @@
 //          block's slice may be written and sent.
 //   barN3  the sums of squares of a block from every CTA of the cluster have landed
 //          (st.async transaction bytes; 3 slots)
+//   barTB, barTX, barZ: TMA of the raw B/C rows, the raw x rows, the z tile
 // Barriers waited two blocks back use two slots, so a waiter never meets a barrier that
 // has moved two phases past the one it expects. The group norm of block k is finished one
 // block late (its gated values wait in TMEM), while the MMA of block k+1 runs; a peer can
