@@ -15,8 +15,8 @@
 //   2. delta = softplus(dt + dt_bias) for the group's heads.
 //   3. state rows (h, p): N/4 lanes each hold one float4 of the row;
 //        h[p][:] = exp(delta A) h[p][:] + delta x'[p] B'[:];  y[p] = h[p][:] . C'[:] + D x'[p]
-//      each lane group loads two rows before using either, and six CTAs per SM keep the
-//      rest of the bytes in flight.
+//      each lane group loads two rows before using either; 16 warps per CTA and three CTAs
+//      per SM keep the rest of the bytes in flight.
 //   4. gated RMSNorm over the group's r*P channels; y written in the activation dtype.
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
@@ -25,10 +25,11 @@
 namespace ssd {
 namespace {
 
-constexpr int kThreads = 256;
-// State rows each lane group loads before computing. Two keep the kernel at 40 registers, so
-// six 256-thread CTAs share an SM: on decode_bf16 that streams the state faster (419 us per
-// step) than four rows at 48 registers and five CTAs (445 us) or eight rows (526 us).
+// 512 threads and two state rows in flight per lane group keep the kernel at about 40
+// registers, three CTAs per SM. Measured on decode_bf16 (B200): 389 us per step, against
+// 418 us with 256 threads (six CTAs per SM), 492 us with 128, and 445 / 526 / 477 us with
+// 256 threads and four / eight / one rows in flight.
+constexpr int kThreads = 512;
 constexpr int kRowsInFlight = 2;
 
 template <typename T, int N>
