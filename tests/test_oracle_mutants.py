@@ -5,6 +5,8 @@ term, a wrong sign or index, a transposed operand) into a temporary directory an
 the pin tests against it: at least one pin must fail. Nothing here touches a GPU.
 """
 import os
+
+import numpy as np
 import subprocess
 import tempfile
 
@@ -73,3 +75,48 @@ def test_mutant_is_caught(name, tmp_path):
             except (AssertionError, ValueError, FloatingPointError, RuntimeError):
                 failures += 1
     assert failures >= 1, f"no pin caught the planted mistake: {name}"
+
+
+# The Python compositions of the oracle (decay, packed sequences on slots): plausible mistakes
+# planted by swapping the function, each of which a pin must catch.
+
+def _decay_without_bias(dt, A, dt_bias):
+    u = np.asarray(dt, np.float64)
+    return np.exp(np.asarray(A, np.float64) * np.log1p(np.exp(u)).sum(axis=1))
+
+
+def _decay_sign_flipped(dt, A, dt_bias):
+    return 1.0 / _real_decay(dt, A, dt_bias)
+
+
+def _decay_last_token_only(dt, A, dt_bias):
+    u = np.asarray(dt, np.float64) + np.asarray(dt_bias, np.float64)
+    return np.exp(np.asarray(A, np.float64) * np.log1p(np.exp(u[:, -1])))
+
+
+_real_decay = oracle.decay
+
+
+@pytest.mark.parametrize("mutant", [_decay_without_bias, _decay_sign_flipped, _decay_last_token_only])
+def test_decay_mutant_is_caught(mutant, monkeypatch):
+    monkeypatch.setattr(oracle, "decay", mutant)
+    with pytest.raises(AssertionError):
+        pins.test_final_state_is_linear_in_the_initial_state_with_the_decay_factor()
+
+
+def _varlen_slots_ignored(d, cu, *args, slot_idx=None, has_init=None, **kw):
+    return _real_varlen(d, cu, *args, slot_idx=None, has_init=has_init, **kw)
+
+
+def _varlen_always_continues(d, cu, *args, slot_idx=None, has_init=None, **kw):
+    return _real_varlen(d, cu, *args, slot_idx=slot_idx, has_init=None, **kw)
+
+
+_real_varlen = oracle.prefill_varlen
+
+
+@pytest.mark.parametrize("mutant", [_varlen_slots_ignored, _varlen_always_continues])
+def test_varlen_mutant_is_caught(mutant, monkeypatch):
+    monkeypatch.setattr(oracle, "prefill_varlen", mutant)
+    with pytest.raises(AssertionError):
+        pins.test_varlen_slots_fresh_starts_and_empty_sequences()
