@@ -11,6 +11,8 @@ Contents
   forms.py       two further, separately written fp64 forms of the scan (the chunked
                  SSD decomposition and the quadratic "dual" matrix form), used only to
                  pin the oracle.
+  backward.py    the backward pass (vector-Jacobian product) of the mixer core in fp64,
+                 pinned against finite differences of the compiled oracle.
 
 Pins: every function here is checked in tests/test_oracle_*.py against closed forms,
 invariants and brute force. The mapping conventions that no page fixes (tap order,
