@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -86,6 +87,15 @@ def decode_bytes(w, batch) -> int:
     state = 2 * batch * H * w.headdim * w.dstate * 4
     conv = 2 * batch * w.xbc_channels * 3 * es
     return state + conv + batch * (3 * HP + 2 * GN + H) * es
+
+
+def backward_bytes(w, batch, seqlen) -> int:
+    """Bytes the backward pass must move with gradients on y only and no initial states:
+    read x, z, B, C, dt and dy once, write dx, dz, dB, dC and ddt once. Parameters and their
+    gradients are ignored."""
+    es = 2 if w.act == "bf16" else 4
+    HP, GN, H = w.d_inner, w.ngroups * w.dstate, w.nheads
+    return batch * seqlen * (2 * (2 * HP + 2 * GN + H) + HP) * es
 
 
 def kernel_bytes(name, w, batch, seqlen) -> int | None:
@@ -495,7 +505,54 @@ def main():
                                "frac": ach / hbm, "traffic": measured_traffic("decode_step"),
                                "algorithmic_bytes_per_launch": db, "peak_source": peak_src}}
 
-    ck = clocks.stop()   # sampled over the prefill, end-to-end and decode timed regions
+    # backward pass of the same prefill (gradient on y only): one call per step
+    bwd = None
+    if not a.no_backward:
+        from hybrid_mamba_ssm_causal_b200.workloads import round_bf16
+        HP, GN, H, Cc = w.d_inner, w.ngroups * w.dstate, w.nheads, w.xbc_channels
+        rng = np.random.default_rng(13)
+        dout = dev_t(round_bf16(rng.standard_normal((w.batch, w.seqlen, HP))).astype(np.float32), True)
+        bws = torch.empty(sm.ssd_mixer_backward_workspace_size(d), dtype=torch.uint8, device=dev)
+        ga = {k: torch.empty(w.batch, w.seqlen, n, dtype=adt, device=dev)
+              for k, n in (("x", HP), ("z", HP), ("B", GN), ("C", GN), ("dt", H))}
+        gp = {k: torch.empty(*shape, dtype=torch.float32, device=dev)
+              for k, shape in (("A", (H,)), ("D", (H,)), ("conv_w", (Cc, 4)), ("conv_b", (Cc,)),
+                               ("dt_bias", (H,)), ("norm_w", (HP,)))}
+
+        def bstep(s):
+            i = sets[s % nsets]["in"]
+            sm.ssd_mixer_backward(d, i["x"], i["z"], i["B"], i["C"], i["dt"], P["A"], P["D"], P["conv_w"],
+                                  P["conv_b"], P["dt_bias"], P["norm_w"], None, None, dout, None, None,
+                                  ga["x"], ga["z"], ga["B"], ga["C"], ga["dt"], gp["A"], gp["D"], gp["conv_w"],
+                                  gp["conv_b"], gp["dt_bias"], gp["norm_w"], None, None, bws)
+
+        for s in range(max(3, a.warmup)):
+            bstep(s)
+        torch.cuda.synchronize()
+        barrier()
+        lib.ssd_mixer_profile_enable(1)
+        lib.ssd_mixer_profile_read(*prof_buffers())
+        n0 = lib.ssd_mixer_launch_count()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for s in range(a.steps):
+            bstep(s)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        blaunch = lib.ssd_mixer_launch_count() - n0
+        bk = read_profile(lib)
+        lib.ssd_mixer_profile_enable(0)
+        bms = rank_max(b0.elapsed_time(b1) / a.steps)
+        bb = backward_bytes(w, w.batch, w.seqlen)
+        ach = bb / (bms * 1e-3) / 1e9
+        bwd = {"workload": f"{w.name} backward: b{w.batch} L{w.seqlen}, gradient on y only, {a.steps} calls",
+               "ms_per_call": bms, "tokens_per_s": job_value(world, w.batch * w.seqlen, bms),
+               "launches_per_call": blaunch / a.steps,
+               "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                            "algorithmic_bytes_per_call": bb, "peak_source": peak_src},
+               "kernels": {k: {"ms_per_call": v[0] / a.steps, "launches": v[1]} for k, v in bk.items()}}
+
+    ck = clocks.stop()   # sampled over the prefill, end-to-end, decode and backward timed regions
     cpu = None
     if rank == 0 and not a.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, dec, a.cpu_seconds)
@@ -512,7 +569,8 @@ def main():
                          "achieved_gbs": step_bytes / (ms * 1e-3) / 1e9,
                          "frac": step_bytes / (ms * 1e-3) / 1e9 / hbm, "peak": hbm},
             "roofline": roofline, "kernels": {k: {"ms_total": v[0], "launches": v[1]} for k, v in per_kernel.items()},
-            "gpu_launches": launches, "e2e": e2e, "decode_workload": decode, "clocks": ck, "cpu_baseline": cpu,
+            "gpu_launches": launches, "e2e": e2e, "decode_workload": decode, "backward": bwd, "clocks": ck,
+            "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

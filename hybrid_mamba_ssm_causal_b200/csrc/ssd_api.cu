@@ -24,6 +24,12 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int
         }
         return w;
     }
+    return simt_workspace_layout(b, L, H, P, G, N, Q, act);
+}
+
+WorkspaceLayout simt_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q, int act)
+{
+    WorkspaceLayout w{};
     const size_t es = act == SSD_BF16 ? 2 : 4;
     const int64_t HP = (int64_t)H * P, Cc = HP + 2 * (int64_t)G * N;
     const int64_t nc = Q > 0 ? (L + Q - 1) / Q : 0;
@@ -35,6 +41,25 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int
     w.states = off; off = align256(off + (size_t)(b * nc * H) * (size_t)P * N * 4);
     w.ypre = off;   off = align256(off + (size_t)(b * L * HP) * 4);
     w.ssp = w.bc_conv = off;
+    w.total = off;
+    return w;
+}
+
+BackwardLayout backward_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int act)
+{
+    BackwardLayout w{};
+    w.fwd = simt_workspace_layout(b, L, H, P, G, N, kBackwardChunk, act);
+    const size_t es = act == SSD_BF16 ? 2 : 4;
+    const int64_t HP = (int64_t)H * P, Cc = HP + 2 * (int64_t)G * N, NB = P / kBackwardRows;
+    size_t off = w.fwd.total;
+    w.y = off;          off = align256(off + (size_t)(b * L * HP) * es);
+    w.final_ssm = off;  off = align256(off + (size_t)(b * H) * (size_t)P * N * 4);
+    w.final_conv = off; off = align256(off + (size_t)(b * Cc) * 3 * es);
+    w.dy = off;         off = align256(off + (size_t)(b * L * HP) * 4);
+    w.dxs = off;        off = align256(off + (size_t)(b * L * HP) * 4);
+    w.dBp = off;        off = align256(off + (size_t)(b * L * H * NB) * (size_t)N * 4);
+    w.dCp = off;        off = align256(off + (size_t)(b * L * H * NB) * (size_t)N * 4);
+    w.ddp = off;        off = align256(off + (size_t)(b * H * NB) * (size_t)L * 4);
     w.total = off;
     return w;
 }
@@ -318,6 +343,85 @@ ssd_status ssd_mixer_decode_step(const ssd_dims* d, const void* x, int64_t x_ld,
     p.ssm_state = ssm_state; p.conv_state = conv_state; p.slot_idx = slot_idx;
     p.y = y; p.y_ld = y_ld;
     if (ssd::launch_decode_step(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+size_t ssd_mixer_backward_workspace_size(const ssd_dims* d)
+{
+    if (check_dims(d, false) != SSD_OK || !ssd::backward_supported(d->headdim, d->dstate)) return 0;
+    return ssd::backward_workspace_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->ngroups, d->dstate, d->act)
+        .total;
+}
+
+ssd_status ssd_mixer_backward(const ssd_dims* d, const void* x, int64_t x_ld, const void* z, int64_t z_ld,
+                              const void* B, int64_t B_ld, const void* C, int64_t C_ld, const void* dt,
+                              int64_t dt_ld, const float* A, const float* D, const float* conv_w,
+                              const float* conv_b, const float* dt_bias, const float* norm_w,
+                              const float* init_ssm_state, const void* init_conv_state, const void* dy,
+                              int64_t dy_ld, const float* dfinal_ssm_state, const float* dfinal_conv_state,
+                              void* dx, int64_t dx_ld, void* dz, int64_t dz_ld, void* dB, int64_t dB_ld, void* dC,
+                              int64_t dC_ld, void* ddt, int64_t ddt_ld, float* dA, float* dD, float* dconv_w,
+                              float* dconv_b, float* ddt_bias, float* dnorm_w, float* dinit_ssm_state,
+                              float* dinit_conv_state, void* workspace, size_t workspace_bytes, void* stream)
+{
+    const ssd_status ds = check_dims(d, false);
+    if (ds != SSD_OK) return ds;
+    if (!ssd::backward_supported(d->headdim, d->dstate)) return SSD_ERR_UNSUPPORTED;
+    if (d->seqlen > 65535LL * 32) return SSD_ERR_UNSUPPORTED;   // token segments of the conv backward
+    const size_t es = d->act == SSD_BF16 ? 2 : 4;
+    const int64_t HP = (int64_t)d->nheads * d->headdim, GN = (int64_t)d->ngroups * d->dstate;
+    if (!A || !D || !conv_w || !conv_b || !dt_bias || !norm_w) return SSD_ERR_INVALID_ARG;
+    if (!dA || !dD || !dconv_w || !dconv_b || !ddt_bias || !dnorm_w) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(conv_w) || (init_ssm_state && !aligned16(init_ssm_state)) ||
+        (init_conv_state && ((uintptr_t)init_conv_state % es)))
+        return SSD_ERR_UNSUPPORTED;
+    const ssd::BackwardLayout wl = ssd::backward_workspace_layout(d->batch, d->seqlen, d->nheads, d->headdim,
+                                                                  d->ngroups, d->dstate, d->act);
+    if (!workspace || workspace_bytes < wl.total || ((uintptr_t)workspace & 255u)) return SSD_ERR_INVALID_ARG;
+    if (d->seqlen > 0 && d->batch > 0) {
+        if (!x || !z || !B || !C || !dt || !dy || !dx || !dz || !dB || !dC || !ddt) return SSD_ERR_INVALID_ARG;
+        if (!row_ok(x, x_ld, HP, es, true) || !row_ok(z, z_ld, HP, es, true) ||
+            !row_ok(B, B_ld, GN, es, true) || !row_ok(C, C_ld, GN, es, true) ||
+            !row_ok(dt, dt_ld, d->nheads, es, false) || !row_ok(dy, dy_ld, HP, es, false) ||
+            !row_ok(dx, dx_ld, HP, es, false) || !row_ok(dz, dz_ld, HP, es, false) ||
+            !row_ok(dB, dB_ld, GN, es, false) || !row_ok(dC, dC_ld, GN, es, false) ||
+            !row_ok(ddt, ddt_ld, d->nheads, es, false))
+            return SSD_ERR_UNSUPPORTED;
+    }
+    ssd::BackwardParams p{};
+    ssd::PrefillParams& f = p.f;
+    f.b = d->batch; f.L = d->seqlen;
+    f.H = d->nheads; f.P = d->headdim; f.G = d->ngroups; f.N = d->dstate; f.K = d->dconv;
+    f.Q = ssd::kBackwardChunk; f.eps = d->eps; f.act = d->act;
+    f.nc = (f.L + f.Q - 1) / f.Q;
+    f.x = x; f.z = z; f.B = B; f.C = C; f.dt = dt;
+    f.x_ld = x_ld; f.z_ld = z_ld; f.B_ld = B_ld; f.C_ld = C_ld; f.dt_ld = dt_ld;
+    f.A = A; f.D = D; f.conv_w = conv_w; f.conv_b = conv_b; f.dt_bias = dt_bias; f.norm_w = norm_w;
+    f.init_ssm = init_ssm_state; f.init_conv = init_conv_state;
+    char* ws = (char*)workspace;
+    f.status = (int*)(ws + wl.fwd.status);
+    f.xbc = ws + wl.fwd.xbc;
+    f.delta = (float*)(ws + wl.fwd.delta);
+    f.lam = (float*)(ws + wl.fwd.lam);
+    f.states = (float*)(ws + wl.fwd.states);
+    f.ypre = (float*)(ws + wl.fwd.ypre);
+    f.ssp = (float*)(ws + wl.fwd.ssp);
+    f.bc_conv = ws + wl.fwd.bc_conv;
+    f.y = ws + wl.y; f.y_ld = HP;
+    f.final_ssm = (float*)(ws + wl.final_ssm);
+    f.final_conv = ws + wl.final_conv;
+    p.dout = dy; p.dout_ld = dy_ld;
+    p.dfinal_ssm = dfinal_ssm_state; p.dfinal_conv = dfinal_conv_state;
+    p.dx = dx; p.dz = dz; p.dB = dB; p.dC = dC; p.ddt = ddt;
+    p.dx_ld = dx_ld; p.dz_ld = dz_ld; p.dB_ld = dB_ld; p.dC_ld = dC_ld; p.ddt_ld = ddt_ld;
+    p.dA = dA; p.dD = dD; p.dconv_w = dconv_w; p.dconv_b = dconv_b; p.ddt_bias = ddt_bias; p.dnorm_w = dnorm_w;
+    p.dinit_ssm = dinit_ssm_state; p.dinit_conv = dinit_conv_state;
+    p.dy = (float*)(ws + wl.dy);
+    p.dxs = (float*)(ws + wl.dxs);
+    p.dBp = (float*)(ws + wl.dBp);
+    p.dCp = (float*)(ws + wl.dCp);
+    p.ddp = (float*)(ws + wl.ddp);
+    if (ssd::launch_backward(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }
 

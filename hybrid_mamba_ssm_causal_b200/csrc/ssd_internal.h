@@ -81,6 +81,43 @@ struct WorkspaceLayout {
 // rows = token rows of one call (b*L, or the packed total of a variable-length call).
 WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int H, int P, int G, int N,
                                          int Q, int act);
+// The CUDA-core path's layout (every intermediate in the workspace), whatever the shape.
+WorkspaceLayout simt_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q, int act);
+
+// ---- backward pass (ssd_backward.cu)
+// Tokens per recompute chunk: the backward reruns the CUDA-core forward with this chunk
+// length and recomputes each chunk's states from the one entering it.
+constexpr int kBackwardChunk = 16;
+// State rows p handled by one CTA of the backward scan (so P / 16 row blocks per head).
+constexpr int kBackwardRows = 16;
+
+struct BackwardParams {
+    PrefillParams f;              // the forward's inputs; its workspace regions (chunk Q = 16)
+    const void* dout;             // [b][L][HP] gradient of y, activation dtype
+    int64_t dout_ld;
+    const float* dfinal_ssm;      // [b][H][P][N] or nullptr
+    const float* dfinal_conv;     // [b][Cc][K-1] or nullptr
+    void *dx, *dz, *dB, *dC, *ddt;   // activation dtype, row strides below
+    int64_t dx_ld, dz_ld, dB_ld, dC_ld, ddt_ld;
+    float *dA, *dD, *dconv_w, *dconv_b, *ddt_bias, *dnorm_w;   // written (zeroed, then summed into)
+    float* dinit_ssm;             // [b][H][P][N] or nullptr
+    float* dinit_conv;            // [b][Cc][K-1] or nullptr
+    // workspace
+    float* dy;                    // [b][L][HP] gradient of y before the gate
+    float* dxs;                   // [b][L][HP] gradient of x'
+    float* dBp;                   // [b][L][H][P/16][N] partial gradients of B' (per head, row block)
+    float* dCp;                   // [b][L][H][P/16][N] partial gradients of C'
+    float* ddp;                   // [b][H][P/16][L] partial gradients of delta
+};
+
+struct BackwardLayout {
+    WorkspaceLayout fwd;          // the recompute forward's regions
+    size_t y, final_ssm, final_conv;   // the recompute forward's outputs (not returned)
+    size_t dy, dxs, dBp, dCp, ddp, total;
+};
+BackwardLayout backward_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int act);
+bool backward_supported(int P, int N);
+cudaError_t launch_backward(const BackwardParams& p, cudaStream_t stream);
 
 // Tensor-core path (ssd_prefill_ws.cu): bf16 activations, P = 64, N = 128, 2 or a multiple
 // of 4 heads per group. It keeps every intermediate on chip; the workspace holds only the

@@ -12,8 +12,10 @@ The entry points keep the C names:
                     workspace, stream=None)
   ssd_mixer_decode_step(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
                         ssm_state, conv_state, slot_idx, y, stream=None)
-plus :func:`prefill` / :func:`decode_step`, which allocate the outputs and workspace
-with torch and call the entry points above.
+  ssd_mixer_backward(dims, <prefill inputs>, dy, dfinal_ssm_state, dfinal_conv_state,
+                     <gradients>, workspace, stream=None)
+plus :func:`prefill` / :func:`decode_step` / :func:`backward`, which allocate the outputs
+and workspace with torch and call the entry points above.
 """
 from __future__ import annotations
 
@@ -33,7 +35,8 @@ SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_d
            "ssd_mixer_workspace_status", "ssd_status_string", "ssd_mixer_version",
            "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read",
            "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
-           "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass")
+           "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass",
+           "ssd_mixer_backward_workspace_size", "ssd_mixer_backward")
 
 
 class SsdError(RuntimeError):
@@ -120,6 +123,11 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_state_pass.argtypes = [I64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                          FP, FP, FP, FP, V]
     lib.ssd_mixer_state_pass.restype = ctypes.c_int
+    lib.ssd_mixer_backward_workspace_size.argtypes = [ctypes.POINTER(_CDims)]
+    lib.ssd_mixer_backward_workspace_size.restype = ctypes.c_size_t
+    lib.ssd_mixer_backward.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 + [FP, P] +
+                                       [P, I64, FP, FP] + [P, I64] * 5 + [FP] * 8 + [P, ctypes.c_size_t, V])
+    lib.ssd_mixer_backward.restype = ctypes.c_int
     lib.ssd_mixer_workspace_status.argtypes = [P, V]
     lib.ssd_mixer_workspace_status.restype = ctypes.c_int
     lib.ssd_status_string.argtypes = [ctypes.c_int]
@@ -153,12 +161,14 @@ def _dev(t, name):
 def _rows(t: torch.Tensor, name: str, rows: int, width: int):
     """Pointer and leading dimension of a [.., rows, width]-shaped activation view whose
     consecutive rows (tokens) are ``ld`` elements apart and whose last dim is unit-stride."""
-    if t.dim() < 2 or t.shape[-1] != width or t.stride(-1) != 1:
-        raise ValueError(f"{name}: expected last dim {width} with unit stride, got {tuple(t.shape)}")
+    if t.dim() < 2 or t.shape[-1] != width:
+        raise ValueError(f"{name}: expected last dim {width}, got {tuple(t.shape)}")
     if t.numel() // width != rows:
         raise ValueError(f"{name}: expected {rows} rows, got {t.numel() // width}")
-    if rows == 0:          # nothing is read or written; any row stride will do
+    if rows == 0:          # nothing is read or written; any strides will do
         return _dev(t, name), width
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name}: last dim must have unit stride")
     ld = t.stride(-2)
     # all leading dims must be an even tiling by ld (token t of row i at (i*L + t) * ld)
     expect = ld
@@ -305,6 +315,37 @@ def ssd_mixer_decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_b
     _check(st, "ssd_mixer_decode_step")
 
 
+def ssd_mixer_backward_workspace_size(dims: Dims) -> int:
+    cd = dims.c()
+    return int(load_library().ssd_mixer_backward_workspace_size(ctypes.byref(cd)))
+
+
+def ssd_mixer_backward(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
+                       init_ssm_state, init_conv_state, dy, dfinal_ssm_state, dfinal_conv_state,
+                       dx, dz, dB, dC, ddt, dA, dD, dconv_w, dconv_b, ddt_bias, dnorm_w,
+                       dinit_ssm_state, dinit_conv_state, workspace, stream=None) -> None:
+    lib = load_library()
+    rows = dims.batch * dims.seqlen
+    HP, GN, H = dims.d_inner, dims.ngroups * dims.dstate, dims.nheads
+    ins = []
+    for t, name, w in ((x, "x", HP), (z, "z", HP), (B, "B", GN), (C, "C", GN), (dt, "dt", H)):
+        ins += list(_rows(t, name, rows, w))
+    outs = []
+    for t, name, w in ((dx, "dx", HP), (dz, "dz", HP), (dB, "dB", GN), (dC, "dC", GN), (ddt, "ddt", H)):
+        outs += list(_rows(t, name, rows, w))
+    pdy, dy_ld = _rows(dy, "dy", rows, HP)
+    cd = dims.c()
+    st = lib.ssd_mixer_backward(
+        ctypes.byref(cd), *ins, _dev(A, "A"), _dev(D, "D"), _dev(conv_w, "conv_w"), _dev(conv_b, "conv_b"),
+        _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"), _dev(init_ssm_state, "init_ssm_state"),
+        _dev(init_conv_state, "init_conv_state"), pdy, dy_ld, _dev(dfinal_ssm_state, "dfinal_ssm_state"),
+        _dev(dfinal_conv_state, "dfinal_conv_state"), *outs, _dev(dA, "dA"), _dev(dD, "dD"),
+        _dev(dconv_w, "dconv_w"), _dev(dconv_b, "dconv_b"), _dev(ddt_bias, "ddt_bias"), _dev(dnorm_w, "dnorm_w"),
+        _dev(dinit_ssm_state, "dinit_ssm_state"), _dev(dinit_conv_state, "dinit_conv_state"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "ssd_mixer_backward")
+
+
 def ssd_mixer_workspace_status(workspace, stream=None) -> int:
     return int(load_library().ssd_mixer_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
 
@@ -332,6 +373,34 @@ def prefill(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
     ssd_mixer_prefill(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,
                       init_ssm_state, init_conv_state, y, fs, fc, ws, stream)
     return y, fs, fc
+
+
+def backward(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w, dy,
+             init_ssm_state=None, init_conv_state=None, dfinal_ssm_state=None, dfinal_conv_state=None,
+             workspace=None, stream=None) -> dict:
+    """Allocate the gradients and (if not given) the workspace, then run
+    :func:`ssd_mixer_backward`. Returns a dict of gradients keyed like the inputs (x, z, B, C,
+    dt, A, D, conv_w, conv_b, dt_bias, norm_w, init_ssm, init_conv)."""
+    dev = x.device
+    b, L, H, P, N, Cc = dims.batch, dims.seqlen, dims.nheads, dims.headdim, dims.dstate, dims.xbc_channels
+    HP, GN, act = dims.d_inner, dims.ngroups * dims.dstate, dims.torch_dtype
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"x": torch.empty(b, L, HP, dtype=act, device=dev), "z": torch.empty(b, L, HP, dtype=act, device=dev),
+         "B": torch.empty(b, L, GN, dtype=act, device=dev), "C": torch.empty(b, L, GN, dtype=act, device=dev),
+         "dt": torch.empty(b, L, H, dtype=act, device=dev), "A": torch.empty(H, **f32), "D": torch.empty(H, **f32),
+         "conv_w": torch.empty(Cc, dims.dconv, **f32), "conv_b": torch.empty(Cc, **f32),
+         "dt_bias": torch.empty(H, **f32), "norm_w": torch.empty(HP, **f32),
+         "init_ssm": torch.empty(b, H, P, N, **f32), "init_conv": torch.empty(b, Cc, dims.dconv - 1, **f32)}
+    if workspace is None:
+        n = ssd_mixer_backward_workspace_size(dims)
+        if n == 0:
+            raise SsdError(SSD_ERR_UNSUPPORTED, "ssd_mixer_backward_workspace_size: unsupported dims")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    ssd_mixer_backward(dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w, init_ssm_state,
+                       init_conv_state, dy, dfinal_ssm_state, dfinal_conv_state, g["x"], g["z"], g["B"], g["C"],
+                       g["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"], g["dt_bias"], g["norm_w"],
+                       g["init_ssm"], g["init_conv"], workspace, stream)
+    return g
 
 
 def decode_step(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias, norm_w,

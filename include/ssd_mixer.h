@@ -269,6 +269,60 @@ SSD_API ssd_status ssd_mixer_prefill_static(const ssd_dims* dims,
                                     float* final_ssm_state, void* final_conv_state,
                                     void* stream);
 
+/* Bytes of device workspace ssd_mixer_backward needs for `dims`; 0 when the dims are
+ * invalid or the shape is one the backward does not run. About (b L (3 HP + Cc/2
+ * + 2 H P N / 16 + 2 H (P/16) N) + b (L/16) H P N) * 4 bytes: the recompute forward's
+ * intermediates with 16-token chunks, and the gradient partial sums. */
+SSD_API size_t ssd_mixer_backward_workspace_size(const ssd_dims* dims);
+
+/* Backward pass of the mixer core: the vector-Jacobian product of ssd_mixer_prefill.
+ * The pages train the Mamba-2 mixer through this scan and test gradient flow through it
+ * (Modalities PR #459, sections "Testing" and "Caveats"). For a scalar loss whose
+ * gradients with respect to the prefill's outputs are dy (for y), dfinal_ssm_state and
+ * dfinal_conv_state, this writes the gradients with respect to every input, parameter and
+ * initial state of a prefill with the same inputs. The forward is recomputed inside the
+ * call (nothing is saved from the training forward); dims->chunk is checked as for
+ * ssd_mixer_prefill but not used.
+ *
+ * Inputs: as ssd_mixer_prefill (same shapes, dtypes, strides and alignment rules; NULL
+ *   initial states are zeros), plus
+ *   dy [b][L][HP] activation dtype, row stride dy_ld;
+ *   dfinal_ssm_state [b][H][P][N] fp32 and dfinal_conv_state [b][Cc][K-1] fp32, or NULL
+ *   when the loss does not depend on the final states.
+ * Outputs (written, not added to):
+ *   dx, dz [b][L][HP], dB, dC [b][L][GN], ddt [b][L][H]: activation dtype, row strides;
+ *   dA, dD, ddt_bias [H], dconv_w [Cc][K], dconv_b [Cc], dnorm_w [HP]: fp32;
+ *   dinit_ssm_state [b][H][P][N] fp32 and dinit_conv_state [b][Cc][K-1] fp32, or NULL
+ *   when not wanted (computed whether or not the initial states were given).
+ * workspace: ssd_mixer_backward_workspace_size(dims) bytes, 256-byte aligned.
+ * Runs on CUDA cores in fp32 for fp32 and bf16 activations, P in {16, 32, 64} and N in
+ * {16, 32, 64, 128}; other shapes return SSD_ERR_UNSUPPORTED, as do rows longer than
+ * 2,097,120 tokens. The parameter gradients are fp32 sums whose order of addition is not
+ * fixed, so they may differ from call to call in the last bits. Outputs must not overlap
+ * inputs or one another. All pointers are device pointers owned by the caller. */
+SSD_API ssd_status ssd_mixer_backward(const ssd_dims* dims,
+                              const void* x, int64_t x_ld,
+                              const void* z, int64_t z_ld,
+                              const void* B, int64_t B_ld,
+                              const void* C, int64_t C_ld,
+                              const void* dt, int64_t dt_ld,
+                              const float* A, const float* D,
+                              const float* conv_w, const float* conv_b,
+                              const float* dt_bias, const float* norm_w,
+                              const float* init_ssm_state, const void* init_conv_state,
+                              const void* dy, int64_t dy_ld,
+                              const float* dfinal_ssm_state, const float* dfinal_conv_state,
+                              void* dx, int64_t dx_ld,
+                              void* dz, int64_t dz_ld,
+                              void* dB, int64_t dB_ld,
+                              void* dC, int64_t dC_ld,
+                              void* ddt, int64_t ddt_ld,
+                              float* dA, float* dD, float* dconv_w, float* dconv_b,
+                              float* ddt_bias, float* dnorm_w,
+                              float* dinit_ssm_state, float* dinit_conv_state,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* Reads the device status word that the prefill kernels keep at the start of
  * `workspace` (written by the last call that used it). Synchronises `stream`.
  * Returns SSD_OK, or SSD_ERR_TIMEOUT if a bounded device-side wait gave up, in

@@ -129,3 +129,35 @@ def test_varlen_rejects_missing_pointers_and_small_workspace(lib):
     assert call_varlen(lib, d, ssm=None) == sm.SSD_ERR_INVALID_ARG
     assert call_varlen(lib, d, ws_bytes=16) == sm.SSD_ERR_INVALID_ARG
     assert call_varlen(lib, d, cu=FAKE + 2) == sm.SSD_ERR_UNSUPPORTED   # cu_seqlens not 4-byte aligned
+
+
+def call_backward(lib, d, ptr=FAKE, ws_bytes=1 << 34, dA=FAKE, dy_ld=None):
+    cd = d.c()
+    HP, GN, H = d.d_inner, d.ngroups * d.dstate, d.nheads
+    rows = [ptr, HP, ptr, HP, ptr, GN, ptr, GN, ptr, H]
+    grads = [FAKE, HP, FAKE, HP, FAKE, GN, FAKE, GN, FAKE, H]
+    return lib.ssd_mixer_backward(ctypes.byref(cd), *rows, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                  FAKE, HP if dy_ld is None else dy_ld, None, None, *grads,
+                                  dA, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, ws_bytes, None)
+
+
+def test_backward_shapes_and_workspace_size(lib):
+    ok = _dims(nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128, seqlen=300)
+    need = lib.ssd_mixer_backward_workspace_size(ctypes.byref(ok.c()))
+    # at least the gradient partial sums and the state entering every 16-token chunk
+    assert need >= 4 * (2 * ok.batch * 300 * 8 * 4 * 128 + ok.batch * 19 * 8 * 64 * 128)
+    for bad in (dict(headdim=128), dict(dconv=3), dict(nheads=3, ngroups=2)):
+        d = _dims(**{**dict(nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128), **bad})
+        assert lib.ssd_mixer_backward_workspace_size(ctypes.byref(d.c())) == 0
+        assert call_backward(lib, d) in (sm.SSD_ERR_UNSUPPORTED, sm.SSD_ERR_INVALID_ARG)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    d = _dims(nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128, seqlen=300)
+    need = lib.ssd_mixer_backward_workspace_size(ctypes.byref(d.c()))
+    assert call_backward(lib, d, ws_bytes=need - 1) == sm.SSD_ERR_INVALID_ARG
+    assert call_backward(lib, d, dA=None) == sm.SSD_ERR_INVALID_ARG
+    assert call_backward(lib, d, ptr=None) == sm.SSD_ERR_INVALID_ARG
+    assert call_backward(lib, d, ptr=FAKE + 2) == sm.SSD_ERR_UNSUPPORTED     # rows not 16-byte aligned
+    assert call_backward(lib, d, dy_ld=d.d_inner - 1) == sm.SSD_ERR_UNSUPPORTED
+    assert call_backward(lib, _dims(seqlen=65535 * 32 + 1)) == sm.SSD_ERR_UNSUPPORTED
