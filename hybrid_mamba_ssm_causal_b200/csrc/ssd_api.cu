@@ -48,7 +48,7 @@ WorkspaceLayout simt_workspace_layout(int64_t b, int64_t L, int H, int P, int G,
 BackwardLayout backward_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int act)
 {
     BackwardLayout w{};
-    w.fwd = simt_workspace_layout(b, L, H, P, G, N, kBackwardChunk, act);
+    w.fwd = simt_workspace_layout(b, L, H, P, G, N, kBackwardForwardChunk, act);
     const size_t es = act == SSD_BF16 ? 2 : 4;
     const int64_t HP = (int64_t)H * P, Cc = HP + 2 * (int64_t)G * N, NB = P / kBackwardRows;
     size_t off = w.fwd.total;
@@ -392,7 +392,7 @@ ssd_status ssd_mixer_backward(const ssd_dims* d, const void* x, int64_t x_ld, co
     ssd::PrefillParams& f = p.f;
     f.b = d->batch; f.L = d->seqlen;
     f.H = d->nheads; f.P = d->headdim; f.G = d->ngroups; f.N = d->dstate; f.K = d->dconv;
-    f.Q = ssd::kBackwardChunk; f.eps = d->eps; f.act = d->act;
+    f.Q = ssd::kBackwardForwardChunk; f.eps = d->eps; f.act = d->act;
     f.nc = (f.L + f.Q - 1) / f.Q;
     f.x = x; f.z = z; f.B = B; f.C = C; f.dt = dt;
     f.x_ld = x_ld; f.z_ld = z_ld; f.B_ld = B_ld; f.C_ld = C_ld; f.dt_ld = dt_ld;

@@ -9,15 +9,17 @@
 // initial states. Nothing is saved from the training forward: it is recomputed.
 //
 // Schedule (all on the caller's stream):
-//   forward    the CUDA-core prefill with 16-token chunks, into the workspace: xBC',
+//   forward    the CUDA-core prefill with 64-token chunks, into the workspace: xBC',
 //              delta, the state entering every chunk, the pre-norm y
 //   norm_gate  one warp per (token, group): dy (gradient of y before the gate) and dz from
 //              dout through the gated RMSNorm; dnorm_w summed per block in shared memory,
 //              then added atomically
 //   scan       one CTA per (row, head, 16 state rows p); each thread owns four elements
-//              H[p][n] of one column n. For each chunk, last to first, it recomputes the
-//              chunk's 16 states from the one entering it (registers), then runs the
-//              recurrence backwards with G the gradient of the state after token t:
+//              H[p][n] of one column n. For each chunk, last to first, it steps the state
+//              entering the chunk to the start of each 16-token sub-chunk; for each
+//              sub-chunk, last to first, it recomputes the sub-chunk's 16 states
+//              (registers), then runs the recurrence backwards with G the gradient of the
+//              state after token t:
 //                G += dy_t (x) C'_t,  dC'_t = H_t^T dy_t,  dx'_t = delta_t G B'_t + D dy_t,
 //                dB'_t = delta_t G^T x'_t,  ddelta_t = A a_t <G, H_{t-1}> + <G, x'_t (x) B'_t>,
 //                dA += delta_t a_t <G, H_{t-1}>,  G <- a_t G       (a_t = exp(delta_t A)).
@@ -37,7 +39,9 @@
 namespace ssd {
 namespace {
 
-constexpr int kQb = kBackwardChunk;   // tokens per recompute chunk
+constexpr int kQf = kBackwardForwardChunk;   // tokens per chunk of the recompute forward
+constexpr int kQb = kBackwardChunk;   // tokens per recompute sub-chunk (states in registers)
+constexpr int kSub = kQf / kQb;       // sub-chunks per chunk
 constexpr int kRows = kBackwardRows;  // state rows per scan CTA
 constexpr int kE = 4;                 // state rows per scan thread (four row groups of four)
 constexpr int kConvSeg = 32;          // tokens per conv-backward thread
@@ -109,13 +113,15 @@ __global__ void __launch_bounds__(256) bwd_norm_gate_kernel(BackwardParams p, in
 // ------------------------------------------------------------------ scan backward
 template <int N>
 struct BwdScanSmem {
+    static constexpr int NT = 4 * N;
     static constexpr int NW = N >= 32 ? N / 32 : 1;   // warps per row group
-    static constexpr int NWARPS = 4 * N / 32;
-    float x[kQb][kRows];        // x' of the chunk's tokens, this CTA's rows
-    float dy[kQb][kRows];       // dy, same
-    float b[kQb][N];            // B' of the head's group
-    float c[kQb][N];            // C'
-    float dl[kQb], al[kQb];     // delta and exp(delta A); 0 and 1 past the end of the row
+    static constexpr int NWARPS = NT / 32;
+    float x[kQf][kRows];        // x' of the chunk's tokens, this CTA's rows
+    float dy[kQf][kRows];       // dy, same
+    float b[kQf][N];            // B' of the head's group
+    float c[kQf][N];            // C'
+    float dl[kQf], al[kQf];     // delta and exp(delta A); 0 and 1 past the end of the row
+    float entry[kSub][kE][NT];  // each thread's state entering each 16-token sub-chunk
     float rc[kQb][4][N];        // per row group: dC' summed over its four rows
     float rb[kQb][4][N];        // per row group: dB' summed over its four rows
     float rx[kQb][kRows][NW];   // dx' summed over one warp's columns
@@ -124,6 +130,9 @@ struct BwdScanSmem {
 };
 
 // Thread tid: column n = tid % N, row group rg = tid / N (rows rg*4 .. rg*4+3 of the CTA's 16).
+// Per 64-token chunk of the forward (last to first): stage it, step the state entering it
+// through the chunk to get the state entering each 16-token sub-chunk, then for each
+// sub-chunk (last to first) recompute its 16 states and run the recurrence backwards.
 template <typename T, int P, int N>
 __global__ void __launch_bounds__(4 * N) bwd_scan_kernel(BackwardParams p)
 {
@@ -150,93 +159,115 @@ __global__ void __launch_bounds__(4 * N) bwd_scan_kernel(BackwardParams p)
     float accA = 0.0f, accD = 0.0f;
 
     for (int64_t ck = f.nc - 1; ck >= 0; --ck) {
-        const int64_t t0 = ck * kQb;
-        const int len = (int)min((int64_t)kQb, L - t0);
+        const int64_t t0 = ck * kQf;
+        const int len = (int)min((int64_t)kQf, L - t0);
         __syncthreads();   // the previous chunk's partial sums have been written out
         // stage the chunk; zeros (delta 0, a 1) past the end of the row make those steps no-ops
-        for (int i = tid; i < kQb * kRows; i += NT) {
+        for (int i = tid; i < kQf * kRows; i += NT) {
             const int t = i / kRows, r = i % kRows;
             const bool in = t < len;
             const int64_t row = bi * L + t0 + t;
             s.x[t][r] = in ? ld_f<T>(xbc + row * Cc + (int64_t)h * P + pr + r) : 0.0f;
             s.dy[t][r] = in ? p.dy[row * HP + (int64_t)h * P + pr + r] : 0.0f;
         }
-        for (int i = tid; i < kQb * N; i += NT) {
+        for (int i = tid; i < kQf * N; i += NT) {
             const int t = i / N, m = i % N;
             const bool in = t < len;
             const int64_t row = bi * L + t0 + t;
             s.b[t][m] = in ? ld_f<T>(xbc + row * Cc + HP + (int64_t)g * N + m) : 0.0f;
             s.c[t][m] = in ? ld_f<T>(xbc + row * Cc + HP + GN + (int64_t)g * N + m) : 0.0f;
         }
-        if (tid < kQb) {
-            const float dl = tid < len ? f.delta[(bi * f.H + h) * L + t0 + tid] : 0.0f;
-            s.dl[tid] = dl;
-            s.al[tid] = expf(dl * A);
+        for (int t = tid; t < kQf; t += NT) {
+            const float dl = t < len ? f.delta[(bi * f.H + h) * L + t0 + t] : 0.0f;
+            s.dl[t] = dl;
+            s.al[t] = expf(dl * A);
         }
-        float hin[kE];
+        float hc[kE];
         const float* st = f.states + ((bi * f.nc + ck) * f.H + h) * PN;
 #pragma unroll
-        for (int e = 0; e < kE; ++e) hin[e] = st[(int64_t)(p0 + e) * N + n];
+        for (int e = 0; e < kE; ++e) hc[e] = st[(int64_t)(p0 + e) * N + n];
         __syncthreads();
-
-        // the chunk's states, recomputed from the state entering it
-        float hs[kQb][kE];
+        // the state entering each 16-token sub-chunk (each thread keeps its own four elements)
+        for (int j = 0; j < kSub; ++j) {
 #pragma unroll
-        for (int t = 0; t < kQb; ++t) {
-            const float a = s.al[t], db = s.dl[t] * s.b[t][n];
+            for (int e = 0; e < kE; ++e) s.entry[j][e][tid] = hc[e];
 #pragma unroll
-            for (int e = 0; e < kE; ++e) hs[t][e] = a * (t ? hs[t - 1][e] : hin[e]) + db * s.x[t][rg * kE + e];
-        }
-        // the recurrence backwards
+            for (int t = j * kQb; t < (j + 1) * kQb; ++t) {
+                const float a = s.al[t], db = s.dl[t] * s.b[t][n];
 #pragma unroll
-        for (int t = kQb - 1; t >= 0; --t) {
-            const float a = s.al[t], dl = s.dl[t], bn = s.b[t][n], cn = s.c[t][n];
-            float pc = 0.0f, gh = 0.0f, gx = 0.0f, px[kE];
-#pragma unroll
-            for (int e = 0; e < kE; ++e) {
-                const float dyv = s.dy[t][rg * kE + e], xv = s.x[t][rg * kE + e];
-                G[e] += dyv * cn;
-                pc += dyv * hs[t][e];
-                gh += G[e] * (t ? hs[t - 1][e] : hin[e]);
-                gx += G[e] * xv;
-                px[e] = dl * G[e] * bn;
+                for (int e = 0; e < kE; ++e) hc[e] = a * hc[e] + db * s.x[t][rg * kE + e];
             }
-            accA += dl * a * gh;
-            s.rc[t][rg][n] = pc;
-            s.rb[t][rg][n] = dl * gx;
+        }
+        for (int j = kSub - 1; j >= 0; --j) {
+            const int tj = j * kQb;                       // first token of the sub-chunk in the chunk
+            const int lj = min(kQb, len - tj);            // its tokens in the row (uniform over the CTA)
+            if (lj <= 0) continue;
+            float hin[kE];
 #pragma unroll
-            for (int e = 0; e < kE; ++e) {   // dx' over the row group's columns (segments of min(N, 32) lanes)
-                float v = px[e];
+            for (int e = 0; e < kE; ++e) hin[e] = s.entry[j][e][tid];
+            // the sub-chunk's states, recomputed from the state entering it
+            float hs[kQb][kE];
 #pragma unroll
-                for (int o = (N < 32 ? N : 32) / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if ((n & 31) == 0) s.rx[t][rg * kE + e][n / 32] = v;
+            for (int t = 0; t < kQb; ++t) {
+                const float a = s.al[tj + t], db = s.dl[tj + t] * s.b[tj + t][n];
+#pragma unroll
+                for (int e = 0; e < kE; ++e)
+                    hs[t][e] = a * (t ? hs[t - 1][e] : hin[e]) + db * s.x[tj + t][rg * kE + e];
             }
-            const float dd = warp_sum(A * a * gh + bn * gx);
-            if (lane == 0) s.rd[t][warp] = dd;
+            // the recurrence backwards
 #pragma unroll
-            for (int e = 0; e < kE; ++e) G[e] *= a;
-        }
-        __syncthreads();
-        // the chunk's sums out: dC', dB' per (head, row block); dx' complete; ddelta per row block
-        for (int i = tid; i < len * N; i += NT) {
-            const int t = i / N, m = i % N;
-            const int64_t o = (((bi * L + t0 + t) * f.H + h) * NB + pb) * N + m;
-            p.dCp[o] = (s.rc[t][0][m] + s.rc[t][1][m]) + (s.rc[t][2][m] + s.rc[t][3][m]);
-            p.dBp[o] = (s.rb[t][0][m] + s.rb[t][1][m]) + (s.rb[t][2][m] + s.rb[t][3][m]);
-        }
-        for (int i = tid; i < len * kRows; i += NT) {
-            const int t = i / kRows, r = i % kRows;
-            float v = Dh * s.dy[t][r];
+            for (int t = kQb - 1; t >= 0; --t) {
+                const int u = tj + t;
+                const float a = s.al[u], dl = s.dl[u], bn = s.b[u][n], cn = s.c[u][n];
+                float pc = 0.0f, gh = 0.0f, gx = 0.0f, px[kE];
 #pragma unroll
-            for (int w = 0; w < S::NW; ++w) v += s.rx[t][r][w];
-            p.dxs[(bi * L + t0 + t) * HP + (int64_t)h * P + pr + r] = v;
-            accD += s.dy[t][r] * s.x[t][r];
-        }
-        if (tid < len) {
-            float v = 0.0f;
+                for (int e = 0; e < kE; ++e) {
+                    const float dyv = s.dy[u][rg * kE + e], xv = s.x[u][rg * kE + e];
+                    G[e] += dyv * cn;
+                    pc += dyv * hs[t][e];
+                    gh += G[e] * (t ? hs[t - 1][e] : hin[e]);
+                    gx += G[e] * xv;
+                    px[e] = dl * G[e] * bn;
+                }
+                accA += dl * a * gh;
+                s.rc[t][rg][n] = pc;
+                s.rb[t][rg][n] = dl * gx;
 #pragma unroll
-            for (int w = 0; w < S::NWARPS; ++w) v += s.rd[tid][w];
-            p.ddp[((bi * f.H + h) * NB + pb) * L + t0 + tid] = v;
+                for (int e = 0; e < kE; ++e) {   // dx' over the row group's columns (segments of min(N, 32) lanes)
+                    float v = px[e];
+#pragma unroll
+                    for (int o = (N < 32 ? N : 32) / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if ((n & 31) == 0) s.rx[t][rg * kE + e][n / 32] = v;
+                }
+                const float dd = warp_sum(A * a * gh + bn * gx);
+                if (lane == 0) s.rd[t][warp] = dd;
+#pragma unroll
+                for (int e = 0; e < kE; ++e) G[e] *= a;
+            }
+            __syncthreads();
+            // the sub-chunk's sums out: dC', dB' per (head, row block); dx' complete; ddelta per row block
+            const int64_t r0 = bi * L + t0 + tj;          // its first token row
+            for (int i = tid; i < lj * N; i += NT) {
+                const int t = i / N, m = i % N;
+                const int64_t o = (((r0 + t) * f.H + h) * NB + pb) * N + m;
+                p.dCp[o] = (s.rc[t][0][m] + s.rc[t][1][m]) + (s.rc[t][2][m] + s.rc[t][3][m]);
+                p.dBp[o] = (s.rb[t][0][m] + s.rb[t][1][m]) + (s.rb[t][2][m] + s.rb[t][3][m]);
+            }
+            for (int i = tid; i < lj * kRows; i += NT) {
+                const int t = i / kRows, r = i % kRows;
+                float v = Dh * s.dy[tj + t][r];
+#pragma unroll
+                for (int w = 0; w < S::NW; ++w) v += s.rx[t][r][w];
+                p.dxs[(r0 + t) * HP + (int64_t)h * P + pr + r] = v;
+                accD += s.dy[tj + t][r] * s.x[tj + t][r];
+            }
+            if (tid < lj) {
+                float v = 0.0f;
+#pragma unroll
+                for (int w = 0; w < S::NWARPS; ++w) v += s.rd[tid][w];
+                p.ddp[((bi * f.H + h) * NB + pb) * L + t0 + tj + tid] = v;
+            }
+            __syncthreads();   // before the next sub-chunk overwrites the partial sums
         }
     }
     if (p.dinit_ssm) {

@@ -85,14 +85,15 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int
 WorkspaceLayout simt_workspace_layout(int64_t b, int64_t L, int H, int P, int G, int N, int Q, int act);
 
 // ---- backward pass (ssd_backward.cu)
-// Tokens per recompute chunk: the backward reruns the CUDA-core forward with this chunk
-// length and recomputes each chunk's states from the one entering it.
+// The backward reruns the CUDA-core forward with 64-token chunks (the state entering each one
+// is kept in the workspace); its scan recomputes the states of a chunk 16 tokens at a time.
+constexpr int kBackwardForwardChunk = 64;
 constexpr int kBackwardChunk = 16;
 // State rows p handled by one CTA of the backward scan (so P / 16 row blocks per head).
 constexpr int kBackwardRows = 16;
 
 struct BackwardParams {
-    PrefillParams f;              // the forward's inputs; its workspace regions (chunk Q = 16)
+    PrefillParams f;              // the forward's inputs; its workspace regions (chunk Q = 64)
     const void* dout;             // [b][L][HP] gradient of y, activation dtype
     int64_t dout_ld;
     const float* dfinal_ssm;      // [b][H][P][N] or nullptr

@@ -270,9 +270,10 @@ SSD_API ssd_status ssd_mixer_prefill_static(const ssd_dims* dims,
                                     void* stream);
 
 /* Bytes of device workspace ssd_mixer_backward needs for `dims`; 0 when the dims are
- * invalid or the shape is one the backward does not run. About (b L (3 HP + Cc/2
- * + 2 H P N / 16 + 2 H (P/16) N) + b (L/16) H P N) * 4 bytes: the recompute forward's
- * intermediates with 16-token chunks, and the gradient partial sums. */
+ * invalid or the shape is one the backward does not run. About (b L (4 HP + Cc + 2 H
+ * (P/16) N + H (P/16) + 2 H) + b (L/64) H P N) * 4 bytes: the recompute forward's
+ * intermediates (the state entering every 64-token chunk among them) and the gradient
+ * partial sums. */
 SSD_API size_t ssd_mixer_backward_workspace_size(const ssd_dims* dims);
 
 /* Backward pass of the mixer core: the vector-Jacobian product of ssd_mixer_prefill.
