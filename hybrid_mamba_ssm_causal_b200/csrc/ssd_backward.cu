@@ -232,12 +232,20 @@ __global__ void __launch_bounds__(4 * N) bwd_scan_kernel(BackwardParams p)
                 accA += dl * a * gh;
                 s.rc[t][rg][n] = pc;
                 s.rb[t][rg][n] = dl * gx;
+                {   // dx': the four rows' sums over the row group's columns, reduce-scattered over a
+                    // segment of min(N, 32) lanes. After the two halving steps a lane keeps one row
+                    // (slot 2 hiA + hiB), summed over its segment by the remaining steps.
+                    constexpr int SEG = N < 32 ? N : 32, O1 = SEG / 2, O2 = SEG / 4;
+                    const bool hiA = (lane & O1) != 0, hiB = (lane & O2) != 0;
+                    float k0 = hiA ? px[2] : px[0], k1 = hiA ? px[3] : px[1];
+                    const float s0 = hiA ? px[0] : px[2], s1 = hiA ? px[1] : px[3];
+                    k0 += __shfl_xor_sync(0xffffffffu, s0, O1);
+                    k1 += __shfl_xor_sync(0xffffffffu, s1, O1);
+                    float k = hiB ? k1 : k0;
+                    k += __shfl_xor_sync(0xffffffffu, hiB ? k0 : k1, O2);
 #pragma unroll
-                for (int e = 0; e < kE; ++e) {   // dx' over the row group's columns (segments of min(N, 32) lanes)
-                    float v = px[e];
-#pragma unroll
-                    for (int o = (N < 32 ? N : 32) / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                    if ((n & 31) == 0) s.rx[t][rg * kE + e][n / 32] = v;
+                    for (int o = O2 / 2; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+                    if ((lane & (O2 - 1)) == 0) s.rx[t][rg * kE + (hiA ? 2 : 0) + (hiB ? 1 : 0)][n / 32] = k;
                 }
                 const float dd = warp_sum(A * a * gh + bn * gx);
                 if (lane == 0) s.rd[t][warp] = dd;
