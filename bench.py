@@ -9,9 +9,10 @@ final states, so every stage of the path runs once per step. ``value`` is tokens
 processed per second (prefill + decode tokens) over all ranks.
 
 The same JSON line carries the decode workload (batch 256, 128 heads x 64, 8 groups,
-d_state 128, fp32 state, 1000 steps) in ``decode_workload``, the dominant kernel's
-roofline, an end-to-end number with host buffers, the clocks seen during the timed
-region and the fp64 CPU oracle timed on the host cores.
+d_state 128, fp32 state, 1000 steps) in ``decode_workload``, the backward pass of the
+step's prefill (gradient on y) in ``backward``, the dominant kernel's roofline, an
+end-to-end number with host buffers, the clocks seen during the timed region and the fp64
+CPU oracle timed on the host cores.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 

@@ -1,7 +1,7 @@
-"""The context-parallel driver's multi-rank logic on CPU: two gloo ranks, each holding one
-piece of a row, run hybrid_mamba_ssm_causal_b200.context_parallel with the kernels replaced by
-the fp64 oracle; the pieces' outputs and the last rank's final states must equal one oracle
-prefill over the whole row."""
+"""The context-parallel driver's multi-rank logic on CPU: two or three gloo ranks, each
+holding one piece of a row, run hybrid_mamba_ssm_causal_b200.context_parallel with the
+kernels replaced by the fp64 oracle; the pieces' outputs and the last rank's final states
+must equal one oracle prefill over the whole row."""
 import os
 import socket
 
@@ -91,16 +91,17 @@ def free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("lens", [(23, 19), (3, 40)])
-def test_two_gloo_ranks_match_one_prefill(lens):
+@pytest.mark.parametrize("lens", [(23, 19), (3, 40), (11, 7, 9)])
+def test_gloo_ranks_match_one_prefill(lens):
+    world = len(lens)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
-    procs = [ctx.Process(target=worker, args=(r, 2, port, lens, q)) for r in range(2)]
+    procs = [ctx.Process(target=worker, args=(r, world, port, lens, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = dict()
-    for _ in range(2):
+    for _ in range(world):
         r, y, fs, fc = q.get(timeout=120)
         res[r] = (y, fs, fc)
     for p in procs:
@@ -109,11 +110,12 @@ def test_two_gloo_ranks_match_one_prefill(lens):
     full, params, init_ssm, init_conv, (b, H, P, G, N) = problem(lens=lens)
     ref = oracle.prefill(oracle.Dims(b, sum(lens), H, P, G, N, 4, 1e-5), *(full[k] for k in SEQ),
                          *(params[k] for k in PAR), init_ssm, init_conv)
-    y = np.concatenate([res[0][0], res[1][0]], axis=1)
+    y = np.concatenate([res[r][0] for r in range(world)], axis=1)
     scale = np.max(np.abs(ref["y"]))
     assert np.max(np.abs(y - ref["y"])) <= 1e-10 * scale
-    assert np.max(np.abs(res[1][1] - ref["final_ssm"])) <= 1e-10 * np.max(np.abs(ref["final_ssm"]))
-    assert np.array_equal(res[1][2], ref["final_conv"])
+    last = res[world - 1]
+    assert np.max(np.abs(last[1] - ref["final_ssm"])) <= 1e-10 * np.max(np.abs(ref["final_ssm"]))
+    assert np.array_equal(last[2], ref["final_conv"])
 
 
 def test_pieces_need_three_tokens():

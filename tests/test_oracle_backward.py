@@ -125,3 +125,26 @@ def test_state_gradients_closed_form_without_output_gradient():
         if L < 3:
             want[:, :, L:] = dfc[:, :, :3 - L]
         assert np.array_equal(g["init_conv"], want)
+
+
+def test_backward_separates_by_group():
+    """The gradients of one group's inputs, of its heads' parameters and of its channels'
+    conv and norm weights are those of the group's own sub-problem (the forward separates by
+    group). The full-size GPU test relies on this to check one group of a large workload."""
+    rng = np.random.default_rng(213)
+    d, inp = rand_problem(rng, b=2, L=23, H=4, P=3, G=2, N=5)
+    dout = rng.standard_normal((2, 23, 12))
+    dfs = rng.standard_normal((2, 4, 3, 5))
+    dfc = rng.standard_normal((2, d.xbc_channels, 3))
+    full = prefill_vjp(d, inp, dout, dfs, dfc)
+    for g in range(d.ngroups):
+        sd, sub, xs, hs, conv_idx = oracle.group_subproblem(d, g, inp)
+        part = prefill_vjp(sd, sub, dout[:, :, xs], dfs[:, hs], dfc[:, conv_idx])
+        bs = slice(g * d.dstate, (g + 1) * d.dstate)
+        pick = {"x": lambda a: a[:, :, xs], "z": lambda a: a[:, :, xs], "B": lambda a: a[:, :, bs],
+                "C": lambda a: a[:, :, bs], "dt": lambda a: a[:, :, hs], "A": lambda a: a[hs], "D": lambda a: a[hs],
+                "conv_w": lambda a: a[conv_idx], "conv_b": lambda a: a[conv_idx], "dt_bias": lambda a: a[hs],
+                "norm_w": lambda a: a[xs], "init_ssm": lambda a: a[:, hs], "init_conv": lambda a: a[:, conv_idx]}
+        for k in KEYS:
+            want = pick[k](full[k])
+            assert np.max(np.abs(part[k] - want)) <= 1e-12 * max(1.0, np.max(np.abs(want))), (g, k)
