@@ -36,7 +36,7 @@ SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_d
            "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read",
            "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
            "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass",
-           "ssd_mixer_backward_workspace_size", "ssd_mixer_backward")
+           "ssd_mixer_backward_workspace_size", "ssd_mixer_backward", "ssd_mixer_selftest_wait")
 
 
 class SsdError(RuntimeError):
@@ -128,6 +128,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_backward.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 + [FP, P] +
                                        [P, I64, FP, FP] + [P, I64] * 5 + [FP] * 8 + [P, ctypes.c_size_t, V])
     lib.ssd_mixer_backward.restype = ctypes.c_int
+    lib.ssd_mixer_selftest_wait.argtypes = [P, ctypes.c_longlong, ctypes.c_int, V]
+    lib.ssd_mixer_selftest_wait.restype = ctypes.c_int
     lib.ssd_mixer_workspace_status.argtypes = [P, V]
     lib.ssd_mixer_workspace_status.restype = ctypes.c_int
     lib.ssd_status_string.argtypes = [ctypes.c_int]
@@ -344,6 +346,12 @@ def ssd_mixer_backward(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, dt_bias
         _dev(dinit_ssm_state, "dinit_ssm_state"), _dev(dinit_conv_state, "dinit_conv_state"),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "ssd_mixer_backward")
+
+
+def ssd_mixer_selftest_wait(workspace, limit_cycles: int, arrive: bool, stream=None) -> None:
+    st = load_library().ssd_mixer_selftest_wait(_dev(workspace, "workspace"), int(limit_cycles), int(bool(arrive)),
+                                                _stream(stream))
+    _check(st, "ssd_mixer_selftest_wait")
 
 
 def ssd_mixer_workspace_status(workspace, stream=None) -> int:

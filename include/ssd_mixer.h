@@ -330,6 +330,17 @@ SSD_API ssd_status ssd_mixer_backward(const ssd_dims* dims,
  * which case that call's outputs are invalid. */
 SSD_API ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream);
 
+/* Self-test of the failure path that every bounded device-side wait in the library takes
+ * (the tensor-core kernels wait on mbarriers for TMA loads, peer copies and tensor-core
+ * commits; each wait gives up after a limit of clock cycles, sets the status word at the
+ * start of the workspace and stops waiting). One thread waits on an mbarrier that nothing
+ * arrives on (arrive = 0) or that it has already arrived on itself (arrive != 0), giving up
+ * after limit_cycles SM clock cycles (0 .. 4e9). Afterwards ssd_mixer_workspace_status on
+ * the same workspace reports SSD_ERR_TIMEOUT (gave up) or SSD_OK. workspace: at least 256
+ * bytes, 256-byte aligned, device memory owned by the caller; only its status word is
+ * written. Launches one single-CTA kernel on `stream`; the context stays usable. */
+SSD_API ssd_status ssd_mixer_selftest_wait(void* workspace, long long limit_cycles, int arrive, void* stream);
+
 /* Number of kernels this library has launched in the process so far (all entry
  * points, all devices). A caller reads it before and after a region to count the
  * library's launches in that region. Not a compute call; thread-safe. */

@@ -161,3 +161,10 @@ def test_backward_rejects_bad_arguments(lib):
     assert call_backward(lib, d, ptr=FAKE + 2) == sm.SSD_ERR_UNSUPPORTED     # rows not 16-byte aligned
     assert call_backward(lib, d, dy_ld=d.d_inner - 1) == sm.SSD_ERR_UNSUPPORTED
     assert call_backward(lib, _dims(seqlen=65535 * 32 + 1)) == sm.SSD_ERR_UNSUPPORTED
+
+
+def test_selftest_wait_rejects_bad_arguments(lib):
+    assert lib.ssd_mixer_selftest_wait(None, 1000, 0, None) == sm.SSD_ERR_INVALID_ARG
+    assert lib.ssd_mixer_selftest_wait(FAKE + 16, 1000, 0, None) == sm.SSD_ERR_INVALID_ARG
+    assert lib.ssd_mixer_selftest_wait(FAKE, -1, 0, None) == sm.SSD_ERR_INVALID_ARG
+    assert lib.ssd_mixer_selftest_wait(FAKE, 4000000001, 0, None) == sm.SSD_ERR_INVALID_ARG
