@@ -40,8 +40,8 @@ SMALL_CASES = [
     ("f32", 2, 203, 4, 16, 2, 32, 64, True),      # ragged tail, two groups, initial states
     ("f32", 1, 77, 2, 32, 1, 64, 32, True),
     ("bf16", 2, 300, 8, 64, 2, 128, 128, True),    # ragged: 2 full chunks + 44 tokens
-    ("bf16", 1, 700, 8, 64, 2, 128, 128, True),    # rows cut in two segments (state-only pass first)
-    ("bf16", 1, 1000, 16, 64, 2, 128, 128, True),  # cut rows, groups wider than one cluster
+    ("bf16", 1, 700, 8, 64, 2, 128, 128, True),    # one row, 5 full blocks + 60 tokens
+    ("bf16", 1, 1000, 16, 64, 2, 128, 128, True),  # groups wider than one cluster (8 heads)
     ("bf16", 1, 517, 4, 32, 1, 64, 256, True),     # Q = 256, ragged
     ("bf16", 3, 64, 8, 64, 4, 64, 64, False),      # exactly one chunk
     ("bf16", 1, 1, 4, 64, 2, 128, 128, True),      # one token

@@ -79,8 +79,8 @@ def test_varlen_all_sequences_empty():
 @pytest.mark.parametrize("b,L", [(2, 333), (1, 600)])
 def test_wide_groups_final_states_may_alias_initial_states(b, L):
     """Plain prefill, bf16, 8 heads per group (two clusters of 4 per group), with the final
-    states written over the initial ones (the second shape would otherwise be cut into two
-    segments)."""
+    states written over the initial ones: the first cluster of a group stages the B/C part
+    of the final conv state, so no cluster overwrites an initial state another still reads."""
     base = WORKLOADS["small_bf16"]
     w = base.with_(batch=b, seqlen=L, nheads=16, headdim=64, ngroups=2, dstate=128, chunk=128,
                    init_ssm_std=0.1, init_conv_std=1.0, seed=55)
