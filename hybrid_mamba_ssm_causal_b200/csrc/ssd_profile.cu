@@ -29,8 +29,13 @@ void profile_begin(const char* name, cudaStream_t st, void** token)
     *token = nullptr;
     if (!g_enabled.load(std::memory_order_relaxed)) return;
     Rec* r = new Rec{name, nullptr, nullptr};
-    if (cudaEventCreate(&r->a) != cudaSuccess || cudaEventCreate(&r->b) != cudaSuccess ||
-        cudaEventRecord(r->a, st) != cudaSuccess) {
+    if (cudaEventCreate(&r->a) != cudaSuccess) {
+        delete r;
+        return;
+    }
+    if (cudaEventCreate(&r->b) != cudaSuccess || cudaEventRecord(r->a, st) != cudaSuccess) {
+        cudaEventDestroy(r->a);
+        if (r->b) cudaEventDestroy(r->b);
         delete r;
         return;
     }
@@ -65,8 +70,8 @@ int ssd_mixer_profile_read(const char** names, double* total_ms, int* launches, 
     int n = 0;
     for (const ssd::Rec& r : recs) {
         float ms = 0.0f;
-        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
-            ms = -1.0f;
+        const bool timed =
+            cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess;
         cudaEventDestroy(r.a);
         cudaEventDestroy(r.b);
         int k = 0;
@@ -78,7 +83,7 @@ int ssd_mixer_profile_read(const char** names, double* total_ms, int* launches, 
             launches[n] = 0;
             ++n;
         }
-        total_ms[k] += ms;
+        if (timed) total_ms[k] += ms;   // a pair that could not be timed still counts as a launch
         launches[k] += 1;
     }
     return n;

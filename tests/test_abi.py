@@ -168,3 +168,15 @@ def test_selftest_wait_rejects_bad_arguments(lib):
     assert lib.ssd_mixer_selftest_wait(FAKE + 16, 1000, 0, None) == sm.SSD_ERR_INVALID_ARG
     assert lib.ssd_mixer_selftest_wait(FAKE, -1, 0, None) == sm.SSD_ERR_INVALID_ARG
     assert lib.ssd_mixer_selftest_wait(FAKE, 4000000001, 0, None) == sm.SSD_ERR_INVALID_ARG
+
+
+def test_profile_accounting_without_launches(lib):
+    import ctypes as C
+    names, ms, cnt = (C.c_char_p * 8)(), (C.c_double * 8)(), (C.c_int * 8)()
+    before = lib.ssd_mixer_launch_count()
+    lib.ssd_mixer_profile_enable(1)
+    assert lib.ssd_mixer_profile_read(names, ms, cnt, 8) == 0     # nothing recorded
+    call_backward(lib, _dims(headdim=128))                         # refused before any launch
+    assert lib.ssd_mixer_profile_read(names, ms, cnt, 8) == 0
+    lib.ssd_mixer_profile_enable(0)
+    assert lib.ssd_mixer_launch_count() == before
