@@ -10,7 +10,7 @@ Contents
                  group RMSNorm (built to liboracle_ssd.so by :func:`build`).
   forms.py       two further, separately written fp64 forms of the scan (the chunked
                  SSD decomposition and the quadratic "dual" matrix form), used only to
-                 pin the oracle.
+                 pin the oracle, and the chunked form of the scan's backward.
   backward.py    the backward pass (vector-Jacobian product) of the mixer core in fp64,
                  pinned against finite differences of the compiled oracle.
 

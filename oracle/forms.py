@@ -21,6 +21,11 @@ Head h reads group h // (H // G).
   M[i, j] = (C_i . B_j) * exp(sum_{k=j+1..i} delta_k A) * delta_j (the "dual",
   attention-like side of the duality) with every segment sum taken by a direct loop.
   It is O(L^3) and meant for tiny L only.
+* :func:`chunked_scan_vjp` is the backward pass of :func:`chunked_scan` written in the
+  same block form (per chunk: products of the chunk's matrices with the decay mask, and
+  a reverse pass over the states entering the chunks), for the tests to hold against the
+  sequential backward in oracle/backward.py. The mixer is trained through this scan
+  (Modalities PR #459, sections "Testing" and "Caveats").
 """
 from __future__ import annotations
 
@@ -95,3 +100,76 @@ def quadratic_scan(xa, Ba, Ca, delta, A, D, H0):
         Hf[h] = acc
     y += D[None, :, None] * xa
     return y, Hf
+
+
+def chunked_scan_vjp(xa, Ba, Ca, delta, A, D, H0, dy, dH_final, Q: int):
+    """Gradients of sum(dy * y_pre) + sum(dH_final * H_final) through :func:`chunked_scan`.
+
+    Per chunk (local tokens i, j; lam the inclusive cumsum of a = delta A; u_j = delta_j x_j;
+    W_ij = exp(lam_i - lam_j) for j <= i; K_ij = C_i . B_j; G the gradient of the state
+    leaving the chunk, H the state entering it):
+      y_i      = sum_j K_ij W_ij u_j + exp(lam_i) H C_i + D x_i
+      H_next   = exp(lam_end) H + sum_j exp(lam_end - lam_j) u_j B_j^T
+    so  du_j   = sum_i K_ij W_ij dy_i + exp(lam_end - lam_j) G B_j
+        dC_i   = sum_j W_ij (dy_i . u_j) B_j + exp(lam_i) H^T dy_i
+        dB_j   = sum_i W_ij (dy_i . u_j) C_i + exp(lam_end - lam_j) G^T u_j
+        dlam_i = sum_j K_ij W_ij (dy_i . u_j) - sum_k K_ki W_ki (dy_k . u_i)
+                 + exp(lam_i) dy_i . (H C_i) - exp(lam_end - lam_i) u_i^T G B_i
+                 + [i = end] (exp(lam_end) <G, H> + sum_j exp(lam_end - lam_j) u_j^T G B_j)
+        da_k   = sum_{i >= k} dlam_i,  ddelta = du . x + A da,  dA = sum delta da,
+        dH     = exp(lam_end) G + sum_i exp(lam_i) dy_i C_i^T   (the previous chunk's G).
+    Shapes as :func:`chunked_scan`; dy [L, H, P]; dH_final [H, P, N] or None.
+    Returns (dxa [L, H, P], dBa [L, G, N], dCa [L, G, N], ddelta [L, H], dA [H], dD [H],
+    dH0 [H, P, N])."""
+    xa, Ba, Ca, delta, dy = (np.asarray(a, dtype=np.float64) for a in (xa, Ba, Ca, delta, dy))
+    A, D = np.asarray(A, np.float64), np.asarray(D, np.float64)
+    L, H, P = xa.shape
+    G, N = Ba.shape[1], Ba.shape[2]
+    grp = _group_of(H, G)
+    starts = list(range(0, L, Q))
+    # the state entering every chunk, per head
+    Hin = np.zeros((len(starts) + 1, H, P, N))
+    Hin[0] = np.asarray(H0, dtype=np.float64)
+    for c, c0 in enumerate(starts):
+        c1 = min(c0 + Q, L)
+        for h in range(H):
+            g = grp[h]
+            lam = np.cumsum(delta[c0:c1, h] * A[h])
+            u = delta[c0:c1, h][:, None] * xa[c0:c1, h, :]
+            S = (u * np.exp(lam[-1] - lam)[:, None]).T @ Ba[c0:c1, g, :]
+            Hin[c + 1, h] = np.exp(lam[-1]) * Hin[c, h] + S
+    dxa, ddelta = np.zeros((L, H, P)), np.zeros((L, H))
+    dBa, dCa = np.zeros((L, G, N)), np.zeros((L, G, N))
+    dA, dD = np.zeros(H), np.sum(dy * xa, axis=(0, 2))
+    Gs = np.zeros((H, P, N)) if dH_final is None else np.array(dH_final, dtype=np.float64)
+    for c in range(len(starts) - 1, -1, -1):
+        c0 = starts[c]
+        c1 = min(c0 + Q, L)
+        q = c1 - c0
+        mask = np.tril(np.ones((q, q), dtype=bool))
+        for h in range(H):
+            g = grp[h]
+            Xc, Bc, Cc, dYc = xa[c0:c1, h, :], Ba[c0:c1, g, :], Ca[c0:c1, g, :], dy[c0:c1, h, :]
+            dl = delta[c0:c1, h]
+            lam = np.cumsum(dl * A[h])
+            u = dl[:, None] * Xc
+            Hc, Gc = Hin[c, h], Gs[h]
+            W = np.where(mask, np.exp(np.where(mask, lam[:, None] - lam[None, :], 0.0)), 0.0)
+            K = Cc @ Bc.T
+            dyu = dYc @ u.T                                   # [i, j] = dy_i . u_j
+            e_i, e_end, e_rest = np.exp(lam), np.exp(lam[-1]), np.exp(lam[-1] - lam)
+            GB = Bc @ Gc.T                                    # [j] = G B_j
+            du = (K * W).T @ dYc + e_rest[:, None] * GB
+            dxa[c0:c1, h, :] = dl[:, None] * du + D[h] * dYc
+            dK = W * dyu
+            dCa[c0:c1, g, :] += dK @ Bc + e_i[:, None] * (dYc @ Hc)
+            dBa[c0:c1, g, :] += dK.T @ Cc + e_rest[:, None] * (u @ Gc)
+            T = K * W * dyu
+            uGB = np.sum(u * GB, axis=1)                      # [j] = u_j^T G B_j
+            dlam = T.sum(axis=1) - T.sum(axis=0) + e_i * np.sum(dYc * (Cc @ Hc.T), axis=1) - e_rest * uGB
+            dlam[-1] += e_end * np.sum(Gc * Hc) + np.sum(e_rest * uGB)
+            da = np.cumsum(dlam[::-1])[::-1]
+            ddelta[c0:c1, h] = np.sum(du * Xc, axis=1) + A[h] * da
+            dA[h] += np.sum(dl * da)
+            Gs[h] = e_end * Gc + (dYc * e_i[:, None]).T @ Cc
+    return dxa, dBa, dCa, ddelta, dA, dD, Gs

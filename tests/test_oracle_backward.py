@@ -148,3 +148,28 @@ def test_backward_separates_by_group():
         for k in KEYS:
             want = pick[k](full[k])
             assert np.max(np.abs(part[k] - want)) <= 1e-12 * max(1.0, np.max(np.abs(want))), (g, k)
+
+
+@pytest.mark.parametrize("Q", [1, 3, 8, 16, 64])
+def test_chunked_backward_form_matches_the_sequential_one(Q):
+    """The scan's backward written in the chunked block form (oracle/forms.py) agrees with
+    the step-by-step backward of the recurrence for every chunk length, ragged tails
+    included: two separately written forms of the same derivative."""
+    from oracle.backward import scan_vjp
+    from oracle.forms import chunked_scan_vjp
+    rng = np.random.default_rng(300 + Q)
+    L, H, P, G, N = 37, 4, 3, 2, 5
+    d, inp = rand_problem(rng, b=1, L=L, H=H, P=P, G=G, N=N)
+    f = forward_saved(d, inp["x"], inp["z"], inp["B"], inp["C"], inp["dt"], inp["A"], inp["D"], inp["conv_w"],
+                      inp["conv_b"], inp["dt_bias"], inp["norm_w"], inp["init_ssm"], inp["init_conv"])
+    r = H // G
+    dy = rng.standard_normal((1, L, H, P))
+    dHf = rng.standard_normal((1, H, P, N))
+    seq = scan_vjp(f["Hs"], f["xs"], f["Bh"], f["Ch"], f["delta"], inp["A"], inp["D"], dy, dHf)
+    dxs, dBh, dCh, ddelta, dA, dD, dH0 = seq
+    want = {"x": dxs[0], "B": dBh[0].reshape(L, G, r, N).sum(axis=2), "C": dCh[0].reshape(L, G, r, N).sum(axis=2),
+            "delta": ddelta[0], "A": dA, "D": dD, "H0": dH0[0]}
+    got = chunked_scan_vjp(f["xs"][0], f["Bh"][0][:, ::r], f["Ch"][0][:, ::r], f["delta"][0], inp["A"], inp["D"],
+                           inp["init_ssm"][0], dy[0], dHf[0], Q)
+    for k, g in zip(("x", "B", "C", "delta", "A", "D", "H0"), got):
+        assert np.max(np.abs(g - want[k])) <= 1e-10 * np.max(np.abs(want[k])), (Q, k)

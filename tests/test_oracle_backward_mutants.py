@@ -53,3 +53,29 @@ def test_backward_mutant_is_caught(name, tmp_path):
     dout, dfs, dfc = cotangents(rng, d, True)
     with pytest.raises(AssertionError):
         check_all_gradients(d, inp, dout, dfs, dfc, rng, vjp=mod.prefill_vjp)
+
+
+FORMS = os.path.join(os.path.dirname(SRC), "forms.py")
+
+CHUNKED_MUTANTS = {
+    "decay-gradient column sums dropped": ("T.sum(axis=1) - T.sum(axis=0)", "T.sum(axis=1)"),
+    "state gradient not decayed across chunks": ("Gs[h] = e_end * Gc +", "Gs[h] = Gc +"),
+    "B' gradient without the chunk-state term": ("dK.T @ Cc + e_rest[:, None] * (u @ Gc)", "dK.T @ Cc"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CHUNKED_MUTANTS))
+def test_chunked_backward_mutant_is_caught(name, tmp_path, monkeypatch):
+    import oracle.forms as forms
+    from tests import test_oracle_backward as tob
+    old, new = CHUNKED_MUTANTS[name]
+    src = open(FORMS).read()
+    assert src.count(old) == 1, f"mutation site not unique: {old!r}"
+    path = tmp_path / "forms_mutant.py"
+    path.write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location("forms_mutant", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(forms, "chunked_scan_vjp", mod.chunked_scan_vjp)
+    with pytest.raises(AssertionError):
+        tob.test_chunked_backward_form_matches_the_sequential_one(8)
