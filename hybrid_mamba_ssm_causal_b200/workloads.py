@@ -71,11 +71,13 @@ WORKLOAD_ORDER = ["tiny_f32", "small_bf16", "mid_bf16", "long_bf16", "decode_bf1
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bf16 value (ties to even); returns float32."""
+    """Round float32 values to the nearest bf16 value (ties to even); returns float32.
+    NaN stays NaN (the rounding carry would otherwise turn a low-payload NaN into Inf)."""
     a = np.ascontiguousarray(a, dtype=np.float32)
     bits = a.view(np.uint32).astype(np.uint64)
     bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
-    return bits.astype(np.uint32).view(np.float32)
+    out = bits.astype(np.uint32).view(np.float32)
+    return np.where(np.isnan(a), a, out)
 
 
 def _act(w: Workload, a: np.ndarray) -> np.ndarray:
