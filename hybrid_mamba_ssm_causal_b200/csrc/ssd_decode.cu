@@ -2,9 +2,8 @@
 //
 // One token per sequence, continuing from the state in the sequence's slot (the
 // one-token-at-a-time decode of gllm PR #86, section "Validation"). The step is
-// memory-bound: the fp32
-// SSM state [H][P][N] of every stepped sequence is read once and written once, which
-// is almost all of the bytes. One CTA owns one (sequence, group): the group's x
+// memory-bound: the fp32 SSM state [H][P][N] of every stepped sequence is read once and
+// written once, which is almost all of the bytes. One CTA owns one (sequence, group): the group's x
 // channels (r = H/G heads), its B and C channels and its norm group, so the conv state
 // of every channel is updated by exactly one thread and the gated RMSNorm needs no
 // cross-CTA exchange.
