@@ -18,7 +18,10 @@ prefill's final state is linear in its initial state, so the pieces can run side
   5. each rank runs the full prefill of its piece from those states (ssd_mixer_prefill).
 
 The last rank's final states are the row's final states. Every arithmetic step runs in the
-library's kernels; this module slices views, calls the collectives and the C ABI. The three
+library's kernels; this module slices views, calls the collectives and the C ABI. The
+state-only pass runs on the tensor-core kernel, so the shapes are its own: bf16
+activations, P = 64, N = 128, 2 or a multiple of 4 heads per group (other shapes raise
+SsdError with SSD_ERR_UNSUPPORTED). The three
 phases are separate functions, so a single process can also run the ranks one phase at a
 time (the collectives are then plain lists).
 """
