@@ -5,6 +5,7 @@ holds the kernels' sources (csrc/), the build script, the ctypes binding
 (:mod:`.ssd_mixer`) and the seeded synthetic workloads (:mod:`.workloads`).
 Importing the package does not load the library; the first call does.
 """
-from .ssd_mixer import (Dims, SsdError, alloc_workspace, decode_step, load_library, prefill,  # noqa: F401
-                        ssd_mixer_decode_step, ssd_mixer_prefill, ssd_mixer_prefill_workspace_size,
-                        ssd_mixer_workspace_status)
+from .ssd_mixer import (Dims, SsdError, alloc_workspace, backward, decode_step, load_library, prefill,  # noqa: F401
+                        ssd_mixer_backward, ssd_mixer_backward_workspace_size, ssd_mixer_decode_step,
+                        ssd_mixer_prefill, ssd_mixer_prefill_state, ssd_mixer_prefill_varlen,
+                        ssd_mixer_prefill_workspace_size, ssd_mixer_state_pass, ssd_mixer_workspace_status)

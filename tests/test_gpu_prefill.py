@@ -15,7 +15,7 @@ import torch
 import oracle
 from hybrid_mamba_ssm_causal_b200 import ssd_mixer as sm
 from hybrid_mamba_ssm_causal_b200.workloads import WORKLOADS, make_prefill_inputs
-from tests.gpu_util import (TOL, assert_close, dims_of, gpu_prefill, oracle_dims, relerr, slice_seq,
+from tests.gpu_util import (TOL, assert_close, dims_of, gpu_prefill, oracle_dims, slice_seq,
                             to_dev)
 
 pytestmark = pytest.mark.gpu

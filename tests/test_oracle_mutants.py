@@ -8,7 +8,6 @@ import os
 
 import numpy as np
 import subprocess
-import tempfile
 
 import pytest
 
