@@ -180,3 +180,20 @@ def test_profile_accounting_without_launches(lib):
     assert lib.ssd_mixer_profile_read(names, ms, cnt, 8) == 0
     lib.ssd_mixer_profile_enable(0)
     assert lib.ssd_mixer_launch_count() == before
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C99 translation unit that takes the address of every declared entry point compiles
+    against include/ssd_mixer.h without warnings and links against the library."""
+    import subprocess
+    names = declared_symbols()
+    src = tmp_path / "use_abi.c"
+    body = "\n".join(f"    (void)&{n};" for n in names)
+    src.write_text('#include "ssd_mixer.h"\nint main(void)\n{\n' + body + "\n    return 0;\n}\n")
+    build_mod.build()
+    lib_dir = os.path.dirname(build_mod.LIB)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(tmp_path / "use_abi"), "-L", lib_dir, "-lssd_mixer",
+           "-Wl,--unresolved-symbols=ignore-in-shared-libs"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
