@@ -69,7 +69,7 @@ extern "C" {
 typedef enum ssd_status {
     SSD_OK = 0,
     SSD_ERR_INVALID_ARG = 1,  /* null pointer, bad size, workspace too small */
-    SSD_ERR_UNSUPPORTED = 2,  /* shape/alignment/dtype this build does not run */
+    SSD_ERR_UNSUPPORTED = 2,  /* shape/alignment/dtype the library does not run */
     SSD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
     SSD_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (status word) */
     SSD_ERR_TOO_LARGE = 5,    /* needs more scratch than the fixed static workspace */
