@@ -1,8 +1,9 @@
 """Context-parallel prefill: one long row split into pieces, one piece per rank.
 
-The pages name context parallelism with Mamba state passing as what the long-context phase
-needs (Modalities PR #459, section "Next steps for production at scale", item "MTP and
-long-context"), and test state passing across a split sequence (section "Testing"). A
+The long-context phase needs the sequence split across GPUs, with the Mamba state handed
+from piece to piece (Modalities PR #459, section "Next steps for production at scale", item
+"MTP and long-context"). The same PR tests a state carried over between the parts of a
+split sequence (section "Testing"). A
 prefill's final state is linear in its initial state, so the pieces can run side by side:
 
   1. each rank runs a 3-token prefill of its piece's last raw tokens to get the conv state its

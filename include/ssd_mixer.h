@@ -134,9 +134,8 @@ SSD_API size_t ssd_mixer_prefill_state_workspace_size(const ssd_dims* dims);
  * the decay of each row's whole piece. A piece of a long sequence then hands its state to the
  * next piece without computing its own outputs first, which is the state passing that a
  * sequence split across devices needs (Modalities PR #459, section "Next steps for
- * production at scale", item "MTP and long-context": the long-context phase wants context
- * parallelism with Mamba state passing; section "Testing": state passing across a split
- * sequence). With S_r the final state of piece r computed from a zero initial state and a_r
+ * production at scale", item "MTP and long-context", on splitting long sequences across
+ * GPUs; section "Testing", on a state carried across the parts of a split sequence). With S_r the final state of piece r computed from a zero initial state and a_r
  * its decay, the state entering piece r+1 is a_r * (state entering piece r) + S_r.
  *
  * Same inputs and state layouts as ssd_mixer_prefill, without z, D and norm_w (C is read

@@ -13,10 +13,10 @@ Head h reads group h // (H // G).
   hybrid Mamba-Transformer MoE architecture", commit notes on ssd.py) names: a
   within-chunk cumulative sum of the log-decays, an intra-chunk causal product, a
   per-chunk state, a sequential pass over chunk states, and the state's contribution
-  to each chunk's outputs. The gllm PR #86 "Reference quirk" paragraph reports that
-  one widely used pure-torch version of this form is off at the first token of every
-  later chunk; the form here must match the sequential recurrence at every position,
-  which the oracle tests check at positions k*Q.
+  to each chunk's outputs. The gllm PR #86 "Reference quirk" paragraph reports a
+  pure-torch version of this form whose error appears where each chunk after the first
+  begins; the form here must match the sequential recurrence at every position, which
+  the oracle tests check at positions k*Q.
 * :func:`quadratic_scan` materialises the whole causal L x L mixing matrix
   M[i, j] = (C_i . B_j) * exp(sum_{k=j+1..i} delta_k A) * delta_j (the "dual",
   attention-like side of the duality) with every segment sum taken by a direct loop.

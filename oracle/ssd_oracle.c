@@ -7,7 +7,7 @@
  * it. It shares no code, header, table or helper with the CUDA path.
  *
  * What it computes: everything between in_proj and out_proj of a Nemotron-H
- * Mamba-2 layer, i.e. the causal conv, the selective SSM scan and the gated norm
+ * Mamba-2 layer: its causal conv, its selective state-space scan and its gated norm
  * that the mixer table of gllm PR #86 "feat(model): Nemotron-H hybrid (Mamba2 +
  * attention + MoE) on the CPU" (section "2. feat(model): Nemotron-H on the CPU",
  * row M) places between the two projections:

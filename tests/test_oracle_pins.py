@@ -184,8 +184,8 @@ def test_sequential_matches_chunked_form(Q):
         yo = out["y_pre"][bi].reshape(d.seqlen, d.nheads, d.headdim)
         assert rel(yo, y) <= 1e-10
         assert rel(out["final_ssm"][bi], Hf) <= 1e-10
-        # the first token of every later chunk (where one pure-torch fallback is known
-        # to be off) must agree just as well
+        # the positions where each chunk after the first begins (where a pure-torch
+        # fallback is reported to err) must agree just as well
         ks = np.arange(Q, d.seqlen, Q)
         if len(ks):
             assert rel(yo[ks], y[ks]) <= 1e-10
