@@ -13,6 +13,8 @@ Contents
                  pin the oracle, and the chunked form of the scan's backward.
   backward.py    the backward pass (vector-Jacobian product) of the mixer core in fp64,
                  pinned against finite differences of the compiled oracle.
+  layer.py       the whole mixer layer (in_proj, the core, out_proj) in fp64: the
+                 computation that fusing the projections with the core must reproduce.
 
 Pins: every function here is checked in tests/test_oracle_*.py against closed forms,
 invariants and brute force. The mapping conventions that no page fixes (tap order,
