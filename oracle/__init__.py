@@ -204,7 +204,8 @@ def decay(dt, A, dt_bias):
     a prefill over these tokens carries its initial SSM state into its final one.
     dt [b, L, H]; returns [b, H]."""
     u = np.asarray(dt, np.float64) + np.asarray(dt_bias, np.float64)
-    delta = np.where(u > 20.0, u, np.log1p(np.exp(np.minimum(u, 20.0))))
+    # softplus(u) = log(1 + e^u) written as max(u, 0) + log1p(e^-|u|): exact for every u, no cutoff
+    delta = np.maximum(u, 0.0) + np.log1p(np.exp(-np.abs(u)))
     return np.exp(np.asarray(A, np.float64) * delta.sum(axis=1))
 
 

@@ -93,14 +93,28 @@ def _decay_last_token_only(dt, A, dt_bias):
     return np.exp(np.asarray(A, np.float64) * np.log1p(np.exp(u[:, -1])))
 
 
+def _decay_softplus_cutoff(dt, A, dt_bias):
+    # softplus(u) replaced by u above 20, a shortcut that drops log1p(e^-u)
+    u = np.asarray(dt, np.float64) + np.asarray(dt_bias, np.float64)
+    delta = np.where(u > 20.0, u, np.log1p(np.exp(np.minimum(u, 20.0))))
+    return np.exp(np.asarray(A, np.float64) * delta.sum(axis=1))
+
+
 _real_decay = oracle.decay
 
 
-@pytest.mark.parametrize("mutant", [_decay_without_bias, _decay_sign_flipped, _decay_last_token_only])
+@pytest.mark.parametrize("mutant", [_decay_without_bias, _decay_sign_flipped, _decay_last_token_only,
+                                    _decay_softplus_cutoff])
 def test_decay_mutant_is_caught(mutant, monkeypatch):
     monkeypatch.setattr(oracle, "decay", mutant)
-    with pytest.raises(AssertionError):
-        pins.test_final_state_is_linear_in_the_initial_state_with_the_decay_factor()
+    caught = 0
+    for pin in (pins.test_final_state_is_linear_in_the_initial_state_with_the_decay_factor,
+                pins.test_decay_equals_the_product_of_the_compiled_oracles_step_factors):
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, "no pin caught the planted mistake in decay()"
 
 
 def _varlen_slots_ignored(d, cu, *args, slot_idx=None, has_init=None, **kw):

@@ -436,3 +436,25 @@ def test_final_state_is_linear_in_the_initial_state_with_the_decay_factor():
     a2 = oracle.decay(p2["dt"], inp["A"], inp["dt_bias"])
     chained = a2[:, :, None, None] * r1["final_ssm"] + r2z["final_ssm"]
     assert np.max(np.abs(chained - with_init["final_ssm"])) <= 1e-12 * np.max(np.abs(with_init["final_ssm"]))
+
+
+def test_decay_equals_the_product_of_the_compiled_oracles_step_factors():
+    """oracle.decay against exp(A * sum_t delta_t) with delta taken from the compiled C oracle's
+    stage output (its own softplus), on steps whose argument dt + dt_bias spans (-40, 40): the
+    large arguments (15 .. 40) are where a shortcut of softplus(u) ~ u would differ from the
+    exact value log(1 + e^u). Small A keeps the product representable at those step sizes."""
+    rng = np.random.default_rng(47)
+    d, inp = rand_problem(rng, b=2, L=24, H=4, P=4, G=2, N=8, init=False)
+    u = np.linspace(-40.0, 40.0, d.batch * d.seqlen * d.nheads).reshape(d.batch, d.seqlen, d.nheads)
+    u[:, :6] = rng.uniform(15.0, 40.0, (d.batch, 6, d.nheads))
+    inp["dt"] = u - inp["dt_bias"]
+    inp["A"] = -np.array([1e-3, 2e-3, 5e-4, 1e-3])
+    out = oracle.prefill_dict(d, inp, stages=True)
+    want = np.exp(inp["A"][None, :] * out["delta"].sum(axis=1))
+    got = oracle.decay(inp["dt"], inp["A"], inp["dt_bias"])
+    assert rel(got, want) <= 1e-13
+    # and the steps in (20, 30), where e^-u is still above half an fp64 ulp of u, carry the
+    # correction log1p(e^-u) that a cutoff at 20 would drop
+    big = (u > 20.0) & (u < 30.0)
+    assert big.any() and np.all(out["delta"][big] > u[big])
+    assert np.all(np.abs(got - want) <= 1e-13 * np.abs(want))
