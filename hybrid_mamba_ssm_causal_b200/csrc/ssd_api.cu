@@ -173,6 +173,7 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     cudaStream_t st = (cudaStream_t)stream;
 
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
+    if (ssd::clear_device_status(p.status, st) != cudaSuccess) return SSD_ERR_CUDA;
     if ((tc ? ssd::launch_prefill_ws(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
         return SSD_ERR_CUDA;
     return SSD_OK;
@@ -229,6 +230,7 @@ ssd_status ssd_mixer_prefill_state(const ssd_dims* d, const void* x, int64_t x_l
     p.status = (int*)(ws + wl.status);
     p.ssp = (float*)(ws + wl.ssp);
     p.bc_conv = ws + wl.bc_conv;
+    if (ssd::clear_device_status(p.status, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::launch_prefill_state_ws(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }
@@ -306,6 +308,7 @@ ssd_status ssd_mixer_prefill_varlen(const ssd_dims* d, const int32_t* cu_seqlens
     p.status = (int*)(ws + wl.status);
     p.ssp = (float*)(ws + wl.ssp);
     p.bc_conv = ws + wl.bc_conv;
+    if (ssd::clear_device_status(p.status, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::launch_prefill_ws(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }
@@ -400,6 +403,7 @@ ssd_status ssd_mixer_backward(const ssd_dims* d, const void* x, int64_t x_ld, co
     f.init_ssm = init_ssm_state; f.init_conv = init_conv_state;
     char* ws = (char*)workspace;
     f.status = (int*)(ws + wl.fwd.status);
+    if (ssd::clear_device_status(f.status, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     f.xbc = ws + wl.fwd.xbc;
     f.delta = (float*)(ws + wl.fwd.delta);
     f.lam = (float*)(ws + wl.fwd.lam);
@@ -433,7 +437,11 @@ ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream)
     if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return SSD_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
-    return v == 0 ? SSD_OK : SSD_ERR_TIMEOUT;
+    switch (v) {
+    case ssd::kDevOk: return SSD_OK;
+    case ssd::kDevTimeout: return SSD_ERR_TIMEOUT;
+    default: return SSD_ERR_DEVICE;
+    }
 }
 
 const char* ssd_status_string(ssd_status s)
@@ -445,6 +453,7 @@ const char* ssd_status_string(ssd_status s)
     case SSD_ERR_CUDA: return "CUDA launch or runtime error";
     case SSD_ERR_TIMEOUT: return "a bounded device-side wait timed out";
     case SSD_ERR_TOO_LARGE: return "problem needs more scratch than the fixed static workspace holds";
+    case SSD_ERR_DEVICE: return "a kernel could not start its work (its shared memory base was misaligned)";
     }
     return "unknown status";
 }

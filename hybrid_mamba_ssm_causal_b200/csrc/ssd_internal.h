@@ -13,6 +13,23 @@
 
 namespace ssd {
 
+// Values of the device status word at the start of a prefill workspace. The host clears it
+// (cudaMemsetAsync on the call's stream) before the call's first kernel; a kernel that meets
+// a failure records its code with set_device_status, and the first failure of a call is kept.
+enum DeviceStatus : int {
+    kDevOk = 0,
+    kDevTimeout = 1,          // a bounded wait (mbarrier, peer copy, tensor-core commit) gave up
+    kDevSmemMisaligned = 2,   // the dynamic shared memory base lacked the alignment the kernel needs
+};
+#ifdef __CUDACC__
+__device__ __forceinline__ void set_device_status(int* status, int code) { atomicCAS(status, 0, code); }
+#endif
+// Clears the status word of a call's workspace on its stream.
+inline cudaError_t clear_device_status(int* status, cudaStream_t st)
+{
+    return cudaMemsetAsync(status, 0, sizeof(int), st);
+}
+
 // Everything one prefill call needs, validated by the ABI layer.
 struct PrefillParams {
     int64_t b, L;        // batch rows, tokens per row

@@ -9,11 +9,16 @@
 // file-scope device array of SSD_MIXER_STATIC_WORKSPACE_BYTES instead.
 //
 // The array is a __device__ variable: in host code its name is only a host-side
-// stand-in, so the device address is fetched once per device with cudaGetSymbolAddress
-// (on the first call on that device, with that device current) and cached. Every call
-// on a device shares the array; the prefill kernels write every scratch byte they read
-// in the same call and reset the status word themselves, so no clearing is needed, but
-// two calls whose work overlaps on the GPU (different streams, no ordering) race on it.
+// stand-in, so its device address is fetched with cudaGetSymbolAddress while the caller's
+// context is current, on the first call in that context, and cached under the context's
+// unique ID (cuCtxGetId never hands out an ID twice in a process, so a context created
+// after cudaDeviceReset, or a caller's own non-primary context, gets its own entry).
+// Every call in a context shares the array; the prefill clears the array's status word
+// on its stream before its first kernel, and its kernels write every other scratch byte
+// they read in the same call, so no other clearing is needed, but two calls whose work
+// overlaps on the GPU (different streams, no ordering) race on it.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "../../include/ssd_mixer.h"
@@ -23,25 +28,78 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_workspace[SSD_MIXER_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_ws_ptr[kMaxDevices] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_static_workspace on the current device (looked up once per device).
+struct DriverFns {
+    CtxGetCurrentFn get_current = nullptr;
+    CtxGetIdFn get_id = nullptr;
+};
+
+// The two driver calls, fetched once through the runtime (no link-time libcuda dependency).
+const DriverFns& driver_fns()
+{
+    static DriverFns fns = []() {
+        DriverFns f;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f.get_id = reinterpret_cast<CtxGetIdFn>(p);
+        return f;
+    }();
+    return fns;
+}
+
+constexpr int kMaxContexts = 256;
+struct CacheEntry {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+std::mutex g_mu;
+CacheEntry g_cache[kMaxContexts];
+int g_ncache = 0;
+
+// ID of the context current on this thread; the runtime's primary context is made current
+// first if none is.
+cudaError_t current_context_id(unsigned long long* id)
+{
+    const DriverFns& f = driver_fns();
+    if (!f.get_current || !f.get_id) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (f.get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    if (!ctx) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaSetDevice(dev);   // initialises and binds the primary context
+        if (e != cudaSuccess) return e;
+        if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+    }
+    return f.get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+
+// Device address of g_static_workspace in the current context (looked up once per context).
 cudaError_t static_workspace(void** out)
 {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    unsigned long long id = 0;
+    cudaError_t e = current_context_id(&id);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_ws_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_workspace);
-        if (e != cudaSuccess) return e;
-        g_ws_ptr[dev] = p;
+    for (int i = 0; i < g_ncache; ++i) {
+        if (g_cache[i].ctx_id == id) {
+            *out = g_cache[i].ptr;
+            return cudaSuccess;
+        }
     }
-    *out = g_ws_ptr[dev];
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return e;
+    if (g_ncache < kMaxContexts) g_cache[g_ncache++] = CacheEntry{id, p};   // else: looked up each call
+    *out = p;
     return cudaSuccess;
 }
 
@@ -68,4 +126,11 @@ extern "C" ssd_status ssd_mixer_prefill_static(
                              dt_bias, norm_w, init_ssm_state, init_conv_state, y, y_ld,
                              final_ssm_state, final_conv_state, ws,
                              (size_t)SSD_MIXER_STATIC_WORKSPACE_BYTES, stream);
+}
+
+extern "C" ssd_status ssd_mixer_prefill_static_status(void* stream)
+{
+    void* ws = nullptr;
+    if (static_workspace(&ws) != cudaSuccess) return SSD_ERR_CUDA;
+    return ssd_mixer_workspace_status(ws, stream);
 }

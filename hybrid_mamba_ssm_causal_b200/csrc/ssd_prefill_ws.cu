@@ -220,10 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     // the swizzled TMA tiles need a 1024-byte aligned base; every CTA sees the same base, so
     // all of them leave here together (before any barrier) if it is not
     if (smem_u32(smem) & 1023u) {
-        if (tid == 0) atomicExch(p.status, 1);
+        if (tid == 0) set_device_status(p.status, kDevSmemMisaligned);
         return;
     }
-    if (blockIdx.x == 0 && tid == 0) *p.status = 0;
     for (int c = tid; c < SROW; c += kThreads) {
         const int64_t ch = staged_channel(c);
         const float4 w = *reinterpret_cast<const float4*>(p.conv_w + ch * 4);
@@ -767,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         for (int i = 0; i < 32; ++i) fs[(int64_t)(chalf * 32 + i) * kN + crow] = H[i];
     }
 
-    if (!ok) atomicExch(p.status, 1);
+    if (!ok) set_device_status(p.status, kDevTimeout);
     fence_before_sync();
     __syncthreads();
     cluster.sync();   // no peer still copies into or arrives on this CTA's shared memory

@@ -22,11 +22,10 @@ __global__ void selftest_wait_kernel(int* status, long long limit, int arrive)
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x != 0) return;
     const uint32_t b = smem_u32(&bar);
-    *status = 0;
     mbar_init(b, 1);
     fence_mbar_init();
     if (arrive) mbar_arrive_local(b);
-    if (!mbar_wait_bounded(b, 0, limit)) atomicExch(status, 1);
+    if (!mbar_wait_bounded(b, 0, limit)) set_device_status(status, kDevTimeout);
 }
 
 }  // namespace
@@ -37,6 +36,7 @@ extern "C" ssd_status ssd_mixer_selftest_wait(void* workspace, long long limit_c
     if (!workspace || ((uintptr_t)workspace & 255u)) return SSD_ERR_INVALID_ARG;
     if (limit_cycles < 0 || limit_cycles > 4000000000LL) return SSD_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
+    if (ssd::clear_device_status((int*)workspace, st) != cudaSuccess) return SSD_ERR_CUDA;
     ssd::LaunchScope ls("selftest_wait", st);
     ssd::selftest_wait_kernel<<<1, 32, 0, st>>>((int*)workspace, limit_cycles, arrive ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;

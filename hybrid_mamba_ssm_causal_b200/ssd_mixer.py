@@ -28,7 +28,7 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libssd_mixer.so")
 
-SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT, SSD_ERR_TOO_LARGE = range(6)
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT, SSD_ERR_TOO_LARGE, SSD_ERR_DEVICE = range(7)
 SSD_MIXER_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 SSD_F32, SSD_BF16 = 0, 1
 SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_decode_step",
@@ -36,7 +36,8 @@ SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_d
            "ssd_mixer_launch_count", "ssd_mixer_profile_enable", "ssd_mixer_profile_read",
            "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
            "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass",
-           "ssd_mixer_backward_workspace_size", "ssd_mixer_backward", "ssd_mixer_selftest_wait")
+           "ssd_mixer_backward_workspace_size", "ssd_mixer_backward", "ssd_mixer_selftest_wait",
+           "ssd_mixer_prefill_static_status")
 
 
 class SsdError(RuntimeError):
@@ -110,6 +111,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_prefill_static.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
                                              [FP, P, P, I64, FP, P, V])
     lib.ssd_mixer_prefill_static.restype = ctypes.c_int
+    lib.ssd_mixer_prefill_static_status.argtypes = [V]
+    lib.ssd_mixer_prefill_static_status.restype = ctypes.c_int
     lib.ssd_mixer_prefill_varlen_workspace_size.argtypes = [ctypes.POINTER(_CDims)]
     lib.ssd_mixer_prefill_varlen_workspace_size.restype = ctypes.c_size_t
     lib.ssd_mixer_prefill_varlen.argtypes = ([ctypes.POINTER(_CDims), P, P, P] + [P, I64] * 5 + [FP] * 6 +
@@ -231,6 +234,11 @@ def ssd_mixer_prefill_static(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, d
         _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
         py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
         _stream(stream)))
+
+
+def ssd_mixer_prefill_static_status(stream=None) -> int:
+    """Status word of the fixed array that ssd_mixer_prefill_static uses (synchronises the stream)."""
+    return int(load_library().ssd_mixer_prefill_static_status(_stream(stream)))
 
 
 def ssd_mixer_prefill_varlen_workspace_size(dims: Dims) -> int:

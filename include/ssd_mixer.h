@@ -73,6 +73,7 @@ typedef enum ssd_status {
     SSD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
     SSD_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (status word) */
     SSD_ERR_TOO_LARGE = 5,    /* needs more scratch than the fixed static workspace */
+    SSD_ERR_DEVICE = 6,       /* a kernel could not start its work (status word) */
 } ssd_status;
 
 typedef enum ssd_dtype {
@@ -249,11 +250,15 @@ SSD_API ssd_status ssd_mixer_decode_step(const ssd_dims* dims,
  * process exits. The library allocates nothing here either.
  *  - Calls needing more scratch than that (ssd_mixer_prefill_workspace_size(dims) >
  *    SSD_MIXER_STATIC_WORKSPACE_BYTES) return SSD_ERR_TOO_LARGE and launch nothing.
- *  - The first call on a device looks up the array's device address (with that device
- *    current) and caches it; make that first call before any stream capture.
- *  - All calls on a device share the one array. Calls that overlap on the GPU (other
- *    streams, no ordering between them) race on it and give wrong results: order them
- *    on one stream or with events. */
+ *  - The first call in a CUDA context (with that context current) looks up the array's
+ *    device address and caches it under the context's unique ID, so a caller's own
+ *    non-primary context, or a context created after cudaDeviceReset, gets its own
+ *    lookup; make the first call in a context before any stream capture.
+ *  - All calls in a context share the one array, which keeps the last call's contents.
+ *    Calls that overlap on the GPU (other streams, no ordering between them) race on it
+ *    and give wrong results: order them on one stream or with events.
+ *  - A bounded device-side wait that gives up is recorded in the array's status word, not
+ *    in the return value: read it with ssd_mixer_prefill_static_status. */
 SSD_API ssd_status ssd_mixer_prefill_static(const ssd_dims* dims,
                                     const void* x, int64_t x_ld,
                                     const void* z, int64_t z_ld,
@@ -267,6 +272,14 @@ SSD_API ssd_status ssd_mixer_prefill_static(const ssd_dims* dims,
                                     void* y, int64_t y_ld,
                                     float* final_ssm_state, void* final_conv_state,
                                     void* stream);
+
+/* Status word of the fixed array that ssd_mixer_prefill_static uses, in the current
+ * context (no counterpart in the pages, like the entry point it serves): the same reading
+ * as ssd_mixer_workspace_status, for the last static call enqueued in this context.
+ * Synchronises `stream`; call it on the stream of that prefill. Returns SSD_OK,
+ * SSD_ERR_TIMEOUT or SSD_ERR_DEVICE as ssd_mixer_workspace_status does, or SSD_ERR_CUDA if
+ * the array's address cannot be looked up. */
+SSD_API ssd_status ssd_mixer_prefill_static_status(void* stream);
 
 /* Bytes of device workspace ssd_mixer_backward needs for `dims`; 0 when the dims are
  * invalid or the shape is one the backward does not run. About (b L (4 HP + Cc + 2 H
@@ -324,9 +337,11 @@ SSD_API ssd_status ssd_mixer_backward(const ssd_dims* dims,
                               void* stream);
 
 /* Reads the device status word that the prefill kernels keep at the start of
- * `workspace` (written by the last call that used it). Synchronises `stream`.
- * Returns SSD_OK, or SSD_ERR_TIMEOUT if a bounded device-side wait gave up, in
- * which case that call's outputs are invalid. */
+ * `workspace` (the last call that used it clears it on its stream before its first kernel,
+ * and its kernels record the first failure). Synchronises `stream`. Returns SSD_OK;
+ * SSD_ERR_TIMEOUT if a bounded device-side wait gave up; SSD_ERR_DEVICE if a kernel found
+ * its dynamic shared memory base misaligned and did no work. In both error cases that
+ * call's outputs are invalid. */
 SSD_API ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream);
 
 /* Self-test of the failure path that every bounded device-side wait in the library takes

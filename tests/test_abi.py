@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for s in range(5):
+    for s in range(7):
         assert lib.ssd_status_string(s)
     assert lib.ssd_mixer_version() >= 100
 
