@@ -74,10 +74,14 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 value (ties to even); returns float32.
     NaN stays NaN (the rounding carry would otherwise turn a low-payload NaN into Inf)."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    bits = a.view(np.uint32).astype(np.uint64)
-    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
-    out = bits.astype(np.uint32).view(np.float32)
-    return np.where(np.isnan(a), a, out)
+    bits = a.view(np.uint32)
+    # in 32-bit arithmetic: only NaN bit patterns can wrap, and those are put back below
+    out = ((bits + np.uint32(0x7FFF) + ((bits >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000))
+    out = out.view(np.float32)
+    nan = np.isnan(a)
+    if nan.any():
+        out = np.where(nan, a, out)
+    return out
 
 
 def _act(w: Workload, a: np.ndarray) -> np.ndarray:

@@ -26,10 +26,15 @@ def test_reference_arm_prints_one_contract_line():
     assert line["impl"] == "reference" and line["dtype"] == "f64" and line["data"] == "synthetic"
     assert line["unit"] == "tokens/s" and line["higher_is_better"] is True and line["vs_baseline"] is None
     assert line["steps"] == 1 and line["warmup"] == 1 and line["value"] > 0
-    # value = tokens per step / seconds per step; the small_bf16 step is 2 x (2048 + 1) tokens
-    assert abs(line["value"] - 2 * 2049 / (line["ms_per_step"] * 1e-3)) <= 1e-6 * line["value"]
-    assert line["config"]["workload"].startswith("small_bf16")
+    # value = tokens per step / seconds per step, each step a bounded sample of the long_bf16
+    # step: the first `tok` tokens of the sequence plus one decode token
+    import re
     cb = line["cpu_baseline"]
+    tok = int(re.search(r"first (\d+) tokens", cb["sample"]).group(1))
+    assert 64 <= tok <= 2048
+    assert abs(line["value"] - (tok + 1) / (line["ms_per_step"] * 1e-3)) <= 1e-6 * line["value"]
+    assert line["config"]["workload"].startswith("long_bf16")
+    assert line["config"]["seq_len"] == 32768
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
