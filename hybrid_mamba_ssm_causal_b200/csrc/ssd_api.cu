@@ -179,6 +179,25 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     return SSD_OK;
 }
 
+int ssd_mixer_prefill_path(const ssd_dims* d)
+{
+    if (check_dims(d, false) != SSD_OK) return SSD_PATH_NONE;
+    return ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups) ? SSD_PATH_TENSOR_CORES
+                                                                                           : SSD_PATH_CUDA_CORES;
+}
+
+ssd_status ssd_mixer_prefill_stage_offsets(const ssd_dims* d, size_t* xbc_act, size_t* delta, size_t* y_pre)
+{
+    if (ssd_mixer_prefill_path(d) != SSD_PATH_CUDA_CORES) return SSD_ERR_UNSUPPORTED;
+    if (!xbc_act || !delta || !y_pre) return SSD_ERR_INVALID_ARG;
+    const ssd::WorkspaceLayout wl = ssd::simt_workspace_layout(d->batch, d->seqlen, d->nheads, d->headdim,
+                                                               d->ngroups, d->dstate, d->chunk, d->act);
+    *xbc_act = wl.xbc;
+    *delta = wl.delta;
+    *y_pre = wl.ypre;
+    return SSD_OK;
+}
+
 size_t ssd_mixer_prefill_state_workspace_size(const ssd_dims* d)
 {
     if (check_dims(d, false) != SSD_OK ||

@@ -37,7 +37,8 @@ SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_d
            "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
            "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass",
            "ssd_mixer_backward_workspace_size", "ssd_mixer_backward", "ssd_mixer_selftest_wait",
-           "ssd_mixer_prefill_static_status")
+           "ssd_mixer_prefill_static_status", "ssd_mixer_prefill_path", "ssd_mixer_prefill_stage_offsets")
+SSD_PATH_NONE, SSD_PATH_CUDA_CORES, SSD_PATH_TENSOR_CORES = range(3)
 
 
 class SsdError(RuntimeError):
@@ -111,6 +112,11 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_prefill_static.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
                                              [FP, P, P, I64, FP, P, V])
     lib.ssd_mixer_prefill_static.restype = ctypes.c_int
+    lib.ssd_mixer_prefill_path.argtypes = [ctypes.POINTER(_CDims)]
+    lib.ssd_mixer_prefill_path.restype = ctypes.c_int
+    SZP = ctypes.POINTER(ctypes.c_size_t)
+    lib.ssd_mixer_prefill_stage_offsets.argtypes = [ctypes.POINTER(_CDims), SZP, SZP, SZP]
+    lib.ssd_mixer_prefill_stage_offsets.restype = ctypes.c_int
     lib.ssd_mixer_prefill_static_status.argtypes = [V]
     lib.ssd_mixer_prefill_static_status.restype = ctypes.c_int
     lib.ssd_mixer_prefill_varlen_workspace_size.argtypes = [ctypes.POINTER(_CDims)]
@@ -234,6 +240,26 @@ def ssd_mixer_prefill_static(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, d
         _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
         py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
         _stream(stream)))
+
+
+def ssd_mixer_prefill_path(dims: Dims) -> int:
+    """SSD_PATH_TENSOR_CORES, SSD_PATH_CUDA_CORES or SSD_PATH_NONE: which kernels a prefill of
+    these dims runs (a host-side query)."""
+    cd = dims.c()
+    return int(load_library().ssd_mixer_prefill_path(ctypes.byref(cd)))
+
+
+def prefill_uses_tensor_cores(dims: Dims) -> bool:
+    return ssd_mixer_prefill_path(dims) == SSD_PATH_TENSOR_CORES
+
+
+def ssd_mixer_prefill_stage_offsets(dims: Dims) -> dict:
+    """Byte offsets of xbc_act, delta and y_pre in the workspace of a CUDA-core prefill."""
+    cd = dims.c()
+    o = [ctypes.c_size_t(0) for _ in range(3)]
+    _check(load_library().ssd_mixer_prefill_stage_offsets(ctypes.byref(cd), *[ctypes.byref(v) for v in o]),
+           "ssd_mixer_prefill_stage_offsets")
+    return {"xbc_act": o[0].value, "delta": o[1].value, "y_pre": o[2].value}
 
 
 def ssd_mixer_prefill_static_status(stream=None) -> int:

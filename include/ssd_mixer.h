@@ -127,6 +127,30 @@ SSD_API ssd_status ssd_mixer_prefill(const ssd_dims* dims,
                              void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* Which kernels ssd_mixer_prefill runs for `dims` (a host-side query; nothing is launched):
+ * SSD_PATH_TENSOR_CORES for bf16 activations with P = 64, N = 128 and 2 or a multiple of 4
+ * heads per group (one fused tcgen05 kernel; intermediates stay on chip, dims->chunk is not
+ * used: the chunked form is evaluated in 128-token blocks); SSD_PATH_CUDA_CORES for the other
+ * supported shapes (fp32 FFMA kernels with dims->chunk-token chunks, intermediates in the
+ * workspace); SSD_PATH_NONE when the dims are invalid or unsupported. */
+typedef enum ssd_path {
+    SSD_PATH_NONE = 0,
+    SSD_PATH_CUDA_CORES = 1,
+    SSD_PATH_TENSOR_CORES = 2,
+} ssd_path;
+SSD_API int ssd_mixer_prefill_path(const ssd_dims* dims);
+
+/* Where a CUDA-core prefill (SSD_PATH_CUDA_CORES) leaves its intermediates in its workspace,
+ * for checking each stage on its own: byte offsets from the workspace start of
+ *   xbc_act [b][L][Cc] activation dtype: SiLU(conv) of [x|B|C];
+ *   delta   [b][H][L] fp32: softplus(dt + dt_bias), head-major;
+ *   y_pre   [b][L][HP] fp32: y = C'.h + D x' before the gate and the norm.
+ * They hold the values of the last call that used the workspace. Returns SSD_OK, or
+ * SSD_ERR_UNSUPPORTED for dims that run on the tensor cores (nothing of this is kept there)
+ * or are invalid; host pointers, written only on SSD_OK. */
+SSD_API ssd_status ssd_mixer_prefill_stage_offsets(const ssd_dims* dims, size_t* xbc_act, size_t* delta,
+                                                   size_t* y_pre);
+
 /* Bytes of device workspace ssd_mixer_prefill_state needs for `dims`; 0 when the dims are
  * invalid or the shape is one the state-only pass does not run. */
 SSD_API size_t ssd_mixer_prefill_state_workspace_size(const ssd_dims* dims);

@@ -197,3 +197,26 @@ def test_header_is_plain_c_and_links(tmp_path):
            "-Wl,--unresolved-symbols=ignore-in-shared-libs"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_prefill_path_query(lib):
+    # bf16, P = 64, N = 128 and 2 or a multiple of 4 heads per group: the tensor-core kernel
+    assert sm.ssd_mixer_prefill_path(_dims(headdim=64, dstate=128, nheads=8, ngroups=2)) == sm.SSD_PATH_TENSOR_CORES
+    assert sm.ssd_mixer_prefill_path(_dims(headdim=64, dstate=128, nheads=4, ngroups=2)) == sm.SSD_PATH_TENSOR_CORES
+    # fp32, other head dims, 3 heads per group: the CUDA-core kernels
+    assert sm.ssd_mixer_prefill_path(_dims(act="f32", headdim=64, dstate=128)) == sm.SSD_PATH_CUDA_CORES
+    assert sm.ssd_mixer_prefill_path(_dims(headdim=32, dstate=128)) == sm.SSD_PATH_CUDA_CORES
+    assert sm.ssd_mixer_prefill_path(_dims(headdim=64, dstate=128, nheads=6, ngroups=2)) == sm.SSD_PATH_CUDA_CORES
+    assert sm.ssd_mixer_prefill_path(_dims(dconv=3)) == sm.SSD_PATH_NONE
+
+
+def test_stage_offsets_follow_the_workspace_layout(lib):
+    d = _dims(act="f32", batch=2, seqlen=100, nheads=4, headdim=16, ngroups=2, dstate=16, chunk=64)
+    off = sm.ssd_mixer_prefill_stage_offsets(d)
+    b, L, H, HP, Cc = 2, 100, 4, 64, 64 + 2 * 32
+    a256 = lambda v: (v + 255) // 256 * 256
+    assert off["xbc_act"] % 256 == 0 and off["xbc_act"] >= 256
+    assert off["delta"] >= a256(off["xbc_act"] + b * L * Cc * 4)
+    assert off["y_pre"] + b * L * HP * 4 <= sm.ssd_mixer_prefill_workspace_size(d)
+    with pytest.raises(sm.SsdError):
+        sm.ssd_mixer_prefill_stage_offsets(_dims(headdim=64, dstate=128, nheads=8, ngroups=2))

@@ -189,7 +189,13 @@ def test_inputs_as_views_of_one_packed_projection():
 
 @pytest.mark.parametrize("act", ["f32", "bf16"])
 def test_chunk_size_invariance(act):
-    w = small(act, 1, 640, 8, 64 if act == "bf16" else 32, 2, 128 if act == "bf16" else 64, 64, True, seed=21)
+    """The chunk length Q is a schedule parameter: the CUDA-core path evaluates the chunked form
+    with exactly Q-token chunks, and every Q gives the sequential recurrence's result. Both
+    cases run that path (fp32, and bf16 with head dim 32, which the tensor-core kernel does not
+    take); the tensor-core kernel always works in 128-token blocks, so Q has nothing to vary
+    there."""
+    w = small(act, 1, 640, 8, 32, 2, 64, 64, True, seed=21)
+    assert not sm.prefill_uses_tensor_cores(dims_of(w))
     inp = make_prefill_inputs(w)
     dv = to_dev(inp, act)
     ref = oracle.prefill_dict(oracle_dims(dims_of(w)), inp)
@@ -244,3 +250,42 @@ def test_zero_tokens_passes_states_through():
     torch.cuda.synchronize()
     assert torch.equal(fs, dv["init_ssm"])
     assert torch.equal(fc, dv["init_conv"])
+
+
+@pytest.mark.parametrize("act", ["f32", "bf16"])
+def test_stages_of_the_cuda_core_path(act):
+    """Per-stage parity: the CUDA-core path's intermediates in its workspace (SiLU(conv) of
+    [x|B|C], delta = softplus(dt + dt_bias), and y before the gate and the norm) against the
+    oracle's stage outputs, so a wrong stage is located by itself and not only through y and the
+    final states. bf16 with head dim 32 runs this path too (the tensor-core kernel keeps its
+    intermediates on chip)."""
+    w = small(act, 2, 203, 4, 32, 2, 32, 64, True, seed=23)
+    d = dims_of(w)
+    assert sm.ssd_mixer_prefill_path(d) == sm.SSD_PATH_CUDA_CORES
+    inp = make_prefill_inputs(w)
+    dv = to_dev(inp, act)
+    ws = sm.alloc_workspace(d)
+    gpu_prefill(d, dv, workspace=ws)
+    torch.cuda.synchronize()
+    off = sm.ssd_mixer_prefill_stage_offsets(d)
+    b, L, H, HP, Cc = w.batch, w.seqlen, w.nheads, w.d_inner, w.xbc_channels
+    adt = torch.bfloat16 if act == "bf16" else torch.float32
+    es = 2 if act == "bf16" else 4
+
+    def view(offset, n, dtype, esize):
+        return ws[offset:offset + n * esize].view(dtype)
+
+    xbc = view(off["xbc_act"], b * L * Cc, adt, es).view(b, L, Cc)
+    delta = view(off["delta"], b * H * L, torch.float32, 4).view(b, H, L).transpose(1, 2)
+    y_pre = view(off["y_pre"], b * L * HP, torch.float32, 4).view(b, L, HP)
+    ref = oracle.prefill_dict(oracle_dims(d), inp, stages=True)
+    assert_close("xbc_act", xbc, ref["xbc_act"], TOL[act])
+    assert_close("delta", delta, ref["delta"], 1e-5)
+    assert_close("y_pre", y_pre, ref["y_pre"], TOL[act])
+
+
+def test_stage_offsets_refused_on_the_tensor_core_path():
+    d = dims_of(WORKLOADS["small_bf16"])
+    assert sm.ssd_mixer_prefill_path(d) == sm.SSD_PATH_TENSOR_CORES
+    with pytest.raises(sm.SsdError):
+        sm.ssd_mixer_prefill_stage_offsets(d)
