@@ -14,14 +14,14 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int
                                          int Q, int act)
 {
     WorkspaceLayout w{};
-    if (prefill_tc_supported(act, P, N, H, G)) {   // everything stays on chip
+    if (prefill_tc_supported(act, P, N, H, G)) {   // the scan's intermediates stay on chip
         w.status = 0;
-        w.xbc = w.delta = w.lam = w.states = w.ypre = w.ssp = w.bc_conv = 256;
-        w.total = 256;
-        if (prefill_tc_split(H, G)) {
-            w.bc_conv = align256(256 + (size_t)(rows * H) * (size_t)prefill_ws_partials_per_head() * 4);
-            w.total = align256(w.bc_conv + (size_t)(b * 2 * G * N) * 3 * 2);
-        }
+        w.xbc = w.delta = w.lam = w.states = w.ypre = 256;
+        w.bcp = 256;
+        size_t off = align256(256 + (size_t)rows * (size_t)(2 * G * N) * 2);
+        w.ssp = off;
+        if (prefill_tc_split(H, G)) off = align256(off + (size_t)(rows * H) * (size_t)prefill_ws_partials_per_head() * 4);
+        w.total = off;
         return w;
     }
     return simt_workspace_layout(b, L, H, P, G, N, Q, act);
@@ -40,7 +40,7 @@ WorkspaceLayout simt_workspace_layout(int64_t b, int64_t L, int H, int P, int G,
     w.lam = off;    off = align256(off + (size_t)(b * H * L) * 4);
     w.states = off; off = align256(off + (size_t)(b * nc * H) * (size_t)P * N * 4);
     w.ypre = off;   off = align256(off + (size_t)(b * L * HP) * 4);
-    w.ssp = w.bc_conv = off;
+    w.ssp = w.bcp = off;
     w.total = off;
     return w;
 }
@@ -169,7 +169,7 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     p.states = (float*)(ws + wl.states);
     p.ypre = (float*)(ws + wl.ypre);
     p.ssp = (float*)(ws + wl.ssp);
-    p.bc_conv = ws + wl.bc_conv;
+    p.bcp = ws + wl.bcp;
     cudaStream_t st = (cudaStream_t)stream;
 
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
@@ -248,7 +248,7 @@ ssd_status ssd_mixer_prefill_state(const ssd_dims* d, const void* x, int64_t x_l
     char* ws = (char*)workspace;
     p.status = (int*)(ws + wl.status);
     p.ssp = (float*)(ws + wl.ssp);
-    p.bc_conv = ws + wl.bc_conv;
+    p.bcp = ws + wl.bcp;
     if (ssd::clear_device_status(p.status, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::launch_prefill_state_ws(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
@@ -326,7 +326,7 @@ ssd_status ssd_mixer_prefill_varlen(const ssd_dims* d, const int32_t* cu_seqlens
     char* ws = (char*)workspace;
     p.status = (int*)(ws + wl.status);
     p.ssp = (float*)(ws + wl.ssp);
-    p.bc_conv = ws + wl.bc_conv;
+    p.bcp = ws + wl.bcp;
     if (ssd::clear_device_status(p.status, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     if (ssd::launch_prefill_ws(p, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
@@ -429,7 +429,7 @@ ssd_status ssd_mixer_backward(const ssd_dims* d, const void* x, int64_t x_ld, co
     f.states = (float*)(ws + wl.fwd.states);
     f.ypre = (float*)(ws + wl.fwd.ypre);
     f.ssp = (float*)(ws + wl.fwd.ssp);
-    f.bc_conv = ws + wl.fwd.bc_conv;
+    f.bcp = ws + wl.fwd.bcp;
     f.y = ws + wl.y; f.y_ld = HP;
     f.final_ssm = (float*)(ws + wl.final_ssm);
     f.final_conv = ws + wl.final_conv;

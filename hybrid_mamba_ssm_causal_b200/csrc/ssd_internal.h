@@ -54,8 +54,7 @@ struct PrefillParams {
     float* states;   // [b][nc][H][P][N] chunk states, then states entering each chunk
     float* ypre;     // [b][L][HP] y before the gate and norm
     float* ssp;      // tensor-core path, groups wider than one cluster: [rows][H][parts] sums of g^2
-    void* bc_conv;   // tensor-core path, groups wider than one cluster: [b][2 GN][K-1] final B/C
-                     // conv state, staged until every cluster of the group has read the initial one
+    void* bcp;       // tensor-core path: [rows][2 GN] bf16, SiLU(conv) of the B and C channels
     // Packed variable-length sequences on state slots (cu_seqlens != nullptr): b sequences,
     // L = total packed tokens, sequence i owns rows cu_seqlens[i] .. cu_seqlens[i+1]-1; its
     // states are the slot slot_idx[i] (identity when null) of init_ssm/init_conv, which
@@ -93,7 +92,7 @@ struct DecodeParams {
 
 // Workspace layout of one prefill call; offsets in bytes, each 256-byte aligned.
 struct WorkspaceLayout {
-    size_t status, xbc, delta, lam, states, ypre, ssp, bc_conv, total;
+    size_t status, xbc, delta, lam, states, ypre, ssp, bcp, total;
 };
 // rows = token rows of one call (b*L, or the packed total of a variable-length call).
 WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int H, int P, int G, int N,
@@ -138,9 +137,9 @@ bool backward_supported(int P, int N);
 cudaError_t launch_backward(const BackwardParams& p, cudaStream_t stream);
 
 // Tensor-core path (ssd_prefill_ws.cu): bf16 activations, P = 64, N = 128, 2 or a multiple
-// of 4 heads per group. It keeps every intermediate on chip; the workspace holds only the
-// status word, plus per-(token, head) partial sums of squares when the group is wider than
-// one cluster (prefill_tc_split).
+// of 4 heads per group. Its workspace holds the status word, SiLU(conv) of the B and C
+// channels (computed once for all heads of a group), and per-(token, head) partial sums of
+// squares when the group is wider than one cluster (prefill_tc_split).
 bool prefill_tc_supported(int act, int P, int N, int H, int G);
 bool prefill_tc_split(int H, int G);
 // The state-only pass on the tensor-core path: final states and decay, no output rows.
