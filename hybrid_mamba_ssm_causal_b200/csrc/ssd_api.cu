@@ -120,14 +120,20 @@ size_t ssd_mixer_prefill_workspace_size(const ssd_dims* d)
         .total;
 }
 
-ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, const void* z,
-                             int64_t z_ld, const void* B, int64_t B_ld, const void* C, int64_t C_ld,
-                             const void* dt, int64_t dt_ld, const float* A, const float* D,
-                             const float* conv_w, const float* conv_b, const float* dt_bias,
-                             const float* norm_w, const float* init_ssm_state,
-                             const void* init_conv_state, void* y, int64_t y_ld,
-                             float* final_ssm_state, void* final_conv_state, void* workspace,
-                             size_t workspace_bytes, void* stream)
+}  // extern "C"
+
+namespace ssd {
+
+// The prefill behind ssd_mixer_prefill. With defer_norm, a tensor-core call whose norm group is
+// wider than a cluster leaves y gated but not normalised and returns, in *out, the parameters
+// whose ssp holds the partial sums of squares; with keep_status the status word is not cleared
+// (the caller cleared it before an earlier kernel of its own).
+ssd_status prefill_call(const ssd_dims* d, const void* x, int64_t x_ld, const void* z, int64_t z_ld, const void* B,
+                        int64_t B_ld, const void* C, int64_t C_ld, const void* dt, int64_t dt_ld, const float* A,
+                        const float* D, const float* conv_w, const float* conv_b, const float* dt_bias,
+                        const float* norm_w, const float* init_ssm_state, const void* init_conv_state, void* y,
+                        int64_t y_ld, float* final_ssm_state, void* final_conv_state, void* workspace,
+                        size_t workspace_bytes, void* stream, bool defer_norm, bool keep_status, PrefillParams* out)
 {
     const ssd_status ds = check_dims(d, false);
     if (ds != SSD_OK) return ds;
@@ -173,10 +179,30 @@ ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, con
     cudaStream_t st = (cudaStream_t)stream;
 
     const bool tc = ssd::prefill_tc_supported(d->act, d->headdim, d->dstate, d->nheads, d->ngroups);
-    if (ssd::clear_device_status(p.status, st) != cudaSuccess) return SSD_ERR_CUDA;
+    p.defer_norm = defer_norm && tc && ssd::prefill_tc_split(d->nheads, d->ngroups);
+    if (!keep_status && ssd::clear_device_status(p.status, st) != cudaSuccess) return SSD_ERR_CUDA;
     if ((tc ? ssd::launch_prefill_ws(p, st) : ssd::launch_prefill_simt(p, st)) != cudaSuccess)
         return SSD_ERR_CUDA;
+    if (out) *out = p;
     return SSD_OK;
+}
+
+}  // namespace ssd
+
+extern "C" {
+
+ssd_status ssd_mixer_prefill(const ssd_dims* d, const void* x, int64_t x_ld, const void* z,
+                             int64_t z_ld, const void* B, int64_t B_ld, const void* C, int64_t C_ld,
+                             const void* dt, int64_t dt_ld, const float* A, const float* D,
+                             const float* conv_w, const float* conv_b, const float* dt_bias,
+                             const float* norm_w, const float* init_ssm_state,
+                             const void* init_conv_state, void* y, int64_t y_ld,
+                             float* final_ssm_state, void* final_conv_state, void* workspace,
+                             size_t workspace_bytes, void* stream)
+{
+    return ssd::prefill_call(d, x, x_ld, z, z_ld, B, B_ld, C, C_ld, dt, dt_ld, A, D, conv_w, conv_b, dt_bias, norm_w,
+                             init_ssm_state, init_conv_state, y, y_ld, final_ssm_state, final_conv_state, workspace,
+                             workspace_bytes, stream, false, false, nullptr);
 }
 
 int ssd_mixer_prefill_path(const ssd_dims* d)

@@ -64,6 +64,9 @@ struct PrefillParams {
     const uint8_t* has_init;
     // state-only pass (ssd_mixer_prefill_state): exp(sum_t delta_t * A) per (row, head), [b][H]
     float* decay;
+    // tensor-core path, groups wider than one cluster: leave y gated but not normalised and keep
+    // the partial sums of squares in the workspace (the caller finishes the norm)
+    bool defer_norm;
 
     SSD_HD int64_t HP() const { return (int64_t)H * P; }
     SSD_HD int64_t GN() const { return (int64_t)G * N; }
@@ -142,6 +145,16 @@ cudaError_t launch_backward(const BackwardParams& p, cudaStream_t stream);
 // squares when the group is wider than one cluster (prefill_tc_split).
 bool prefill_tc_supported(int act, int P, int N, int H, int G);
 bool prefill_tc_split(int H, int G);
+// scale[row][g] of the group norm from the partial sums a deferred-norm prefill left in p.ssp.
+cudaError_t launch_norm_scale(const PrefillParams& p, float* scale, cudaStream_t stream);
+
+// The layer's projections (ssd_gemm.cu): C[M][N] = A[M][K] . W[N][K]^T, bf16 in and out, fp32
+// accumulation. With row_scale, A[t][k] is first multiplied by row_scale[t][k / scale_group]
+// (and by col_scale[k] when given), scale_group a multiple of 64.
+bool gemm_supported(int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldw, int64_t ldc);
+cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, const void* W, int64_t ldw,
+                             void* C, int64_t ldc, const float* row_scale, int scale_group, int64_t scale_ld,
+                             const float* col_scale, int* status, cudaStream_t st);
 // The state-only pass on the tensor-core path: final states and decay, no output rows.
 cudaError_t launch_prefill_state_ws(const PrefillParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream);

@@ -916,6 +916,24 @@ __global__ void __launch_bounds__(256) ws_norm_finish_kernel(PrefillParams p)
     }
 }
 
+// The group RMS scale of every (token, group) from the SPLIT kernel's partial sums, for a
+// caller that applies the norm itself (the out_proj prologue of the mixer layer):
+// scale[row][g] = 1 / sqrt(mean over the group of g^2 + eps).
+__global__ void __launch_bounds__(256) ws_norm_scale_kernel(PrefillParams p, float* scale)
+{
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= p.rows() * p.G) return;
+    const int64_t row = w / p.G;
+    const int g = (int)(w % p.G);
+    const int rpg = p.H / p.G, gs = rpg * kP;
+    const float* sp = p.ssp + (row * p.H + (int64_t)g * rpg) * 2;
+    float s = 0.0f;
+    for (int k = lane; k < 2 * rpg; k += 32) s += sp[k];
+    s = warp_sum(s);
+    if (lane == 0) scale[w] = rsqrtf(s / (float)gs + p.eps);
+}
+
 // cuTensorMapEncodeTiled, fetched once through the runtime (no link-time libcuda dependency).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1011,7 +1029,7 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
         e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT, STATE_ONLY>, p, maps);
         if (e != cudaSuccess) return e;
     }
-    if (SPLIT && !STATE_ONLY && p.rows() > 0) {
+    if (SPLIT && !STATE_ONLY && p.rows() > 0 && !p.defer_norm) {
         LaunchScope ls("tc_norm_finish", st);
         const int64_t warps = p.rows() * p.G;
         ws_norm_finish_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
@@ -1042,6 +1060,15 @@ cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream)
 }
 
 int prefill_ws_partials_per_head() { return 2; }
+
+cudaError_t launch_norm_scale(const PrefillParams& p, float* scale, cudaStream_t stream)
+{
+    if (p.rows() == 0) return cudaSuccess;
+    LaunchScope ls("tc_norm_scale", stream);
+    const int64_t warps = p.rows() * p.G;
+    ws_norm_scale_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(p, scale);
+    return cudaGetLastError();
+}
 
 bool prefill_tc_supported(int act, int P, int N, int H, int G)
 {

@@ -113,6 +113,17 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzled layout: rows of
+// 64 bf16 (128 bytes) in 8-row, 1024-byte atoms whose 16-byte chunks are permuted by row % 8
+// (what a TMA load with 128-byte swizzling writes). Stride between 8-row groups 1024 bytes; the
+// leading offset is unused for this layout. Successive K=16 slices of a 64-wide K block start
+// 32 bytes apart. Atoms must start 1024-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulation.
 // a_mn / b_mn: 1 = MN-major operand, 0 = K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn)

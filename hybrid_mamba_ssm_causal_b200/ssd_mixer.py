@@ -37,7 +37,8 @@ SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_d
            "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
            "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass",
            "ssd_mixer_backward_workspace_size", "ssd_mixer_backward", "ssd_mixer_selftest_wait",
-           "ssd_mixer_prefill_static_status", "ssd_mixer_prefill_path", "ssd_mixer_prefill_stage_offsets")
+           "ssd_mixer_prefill_static_status", "ssd_mixer_prefill_path", "ssd_mixer_prefill_stage_offsets",
+           "ssd_mixer_projection", "ssd_mixer_layer_workspace_size", "ssd_mixer_layer_prefill")
 SSD_PATH_NONE, SSD_PATH_CUDA_CORES, SSD_PATH_TENSOR_CORES = range(3)
 
 
@@ -112,6 +113,13 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_prefill_static.argtypes = ([ctypes.POINTER(_CDims)] + [P, I64] * 5 + [FP] * 6 +
                                              [FP, P, P, I64, FP, P, V])
     lib.ssd_mixer_prefill_static.restype = ctypes.c_int
+    lib.ssd_mixer_projection.argtypes = [I64, I64, I64, P, I64, P, I64, P, I64, P, V]
+    lib.ssd_mixer_projection.restype = ctypes.c_int
+    lib.ssd_mixer_layer_workspace_size.argtypes = [ctypes.POINTER(_CDims), I64]
+    lib.ssd_mixer_layer_workspace_size.restype = ctypes.c_size_t
+    lib.ssd_mixer_layer_prefill.argtypes = ([ctypes.POINTER(_CDims), I64, P, I64, P, P] + [FP] * 6 +
+                                            [FP, P, P, I64, FP, P, P, ctypes.c_size_t, V])
+    lib.ssd_mixer_layer_prefill.restype = ctypes.c_int
     lib.ssd_mixer_prefill_path.argtypes = [ctypes.POINTER(_CDims)]
     lib.ssd_mixer_prefill_path.restype = ctypes.c_int
     SZP = ctypes.POINTER(ctypes.c_size_t)
@@ -240,6 +248,58 @@ def ssd_mixer_prefill_static(dims: Dims, x, z, B, C, dt, A, D, conv_w, conv_b, d
         _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"),
         py, y_ld, _dev(final_ssm_state, "final_ssm_state"), _dev(final_conv_state, "final_conv_state"),
         _stream(stream)))
+
+
+def ssd_mixer_projection(A, W, C, workspace, stream=None) -> None:
+    """C = A . W^T on the tensor cores: A [M, K], W [N, K], C [M, N], bf16 (row strides from the
+    tensors; last dims unit-stride). workspace: >= 256 bytes for the status word."""
+    M, K = A.shape[-2], A.shape[-1]
+    N = W.shape[0]
+    for t, nm in ((A, "A"), (W, "W"), (C, "C")):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError(f"{nm}: bf16 with unit-stride rows expected")
+    st = load_library().ssd_mixer_projection(M, N, K, _dev(A, "A"), A.stride(-2), _dev(W, "W"), W.stride(-2),
+                                             _dev(C, "C"), C.stride(-2), _dev(workspace, "workspace"), _stream(stream))
+    _check(st, "ssd_mixer_projection")
+
+
+def ssd_mixer_layer_workspace_size(dims: Dims, d_model: int) -> int:
+    cd = dims.c()
+    return int(load_library().ssd_mixer_layer_workspace_size(ctypes.byref(cd), d_model))
+
+
+def layer_prefill(dims: Dims, hidden, W_in, W_out, A, D, conv_w, conv_b, dt_bias, norm_w,
+                  init_ssm_state=None, init_conv_state=None, workspace=None, out=None, stream=None):
+    """The whole mixer layer (in_proj, the core, out_proj) through ssd_mixer_layer_prefill.
+    hidden [b, L, d_model] bf16; W_in [2HP + 2GN + H, d_model]; W_out [d_model, HP].
+    Returns (out [b, L, d_model], final_ssm_state, final_conv_state)."""
+    lib = load_library()
+    d_model = hidden.shape[-1]
+    rows = dims.batch * dims.seqlen
+    ph, hld = _rows(hidden, "hidden", rows, d_model)
+    dev = hidden.device
+    if workspace is None:
+        n = ssd_mixer_layer_workspace_size(dims, d_model)
+        if n == 0:
+            raise SsdError(SSD_ERR_UNSUPPORTED, "ssd_mixer_layer_workspace_size: unsupported dims")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    if out is None:
+        y = torch.empty(dims.batch, dims.seqlen, d_model, dtype=torch.bfloat16, device=dev)
+        fs = torch.empty(dims.batch, dims.nheads, dims.headdim, dims.dstate, dtype=torch.float32, device=dev)
+        fc = torch.empty(dims.batch, dims.d_inner + 2 * dims.ngroups * dims.dstate, dims.dconv - 1,
+                         dtype=torch.bfloat16, device=dev)
+    else:
+        y, fs, fc = out
+    py, yld = _rows(y, "out", rows, d_model)
+    cd = dims.c()
+    st = lib.ssd_mixer_layer_prefill(
+        ctypes.byref(cd), d_model, ph, hld, _dev(W_in, "W_in"), _dev(W_out, "W_out"), _dev(A, "A"), _dev(D, "D"),
+        _dev(conv_w, "conv_w"), _dev(conv_b, "conv_b"), _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"),
+        _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"), py, yld,
+        _dev(fs, "final_ssm_state"), _dev(fc, "final_conv_state"), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "ssd_mixer_layer_prefill")
+    return y, fs, fc
 
 
 def ssd_mixer_prefill_path(dims: Dims) -> int:

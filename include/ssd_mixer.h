@@ -305,6 +305,51 @@ SSD_API ssd_status ssd_mixer_prefill_static(const ssd_dims* dims,
  * the array's address cannot be looked up. */
 SSD_API ssd_status ssd_mixer_prefill_static_status(void* stream);
 
+/* One projection of the mixer layer on the tensor cores: C[M][N] = A[M][K] . W[N][K]^T, bf16
+ * inputs and output with fp32 accumulation (in_proj maps the block's hidden state to the packed
+ * [z | x | B | C | dt] row, out_proj maps y back to the model width: gllm PR #86 "feat(model):
+ * Nemotron-H hybrid (Mamba2 + attention + MoE) on the CPU", section "2. feat(model): Nemotron-H
+ * on the CPU", mixer table row M). A [M][K] with row stride lda, W [N][K] (the row-major weight
+ * of an N-output linear map) with row stride ldw, C [M][N] with row stride ldc, all in elements;
+ * K and the strides multiples of 8, pointers 16-byte aligned; M, N, K below 2^31. workspace:
+ * 256 device bytes, 256-byte aligned, for the status word (ssd_mixer_workspace_status). Returns
+ * SSD_ERR_UNSUPPORTED for other sizes or alignments. Device pointers owned by the caller; C must
+ * not overlap A or W. */
+SSD_API ssd_status ssd_mixer_projection(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                                        const void* W, int64_t ldw, void* C, int64_t ldc,
+                                        void* workspace, void* stream);
+
+/* Bytes of device workspace ssd_mixer_layer_prefill needs; 0 when the dims or d_model are
+ * invalid or unsupported. */
+SSD_API size_t ssd_mixer_layer_workspace_size(const ssd_dims* dims, int64_t d_model);
+
+/* The whole mixer layer for a prefill: out = out_proj(core(in_proj(hidden))), the pages'
+ * in_proj -> CausalConv1D -> SSMScan -> GatedRMSNorm -> out_proj (gllm PR #86, section "2.
+ * feat(model): Nemotron-H on the CPU", mixer table row M). in_proj emits one packed row per token,
+ * split [z | x | B | C | dt] (gllm PR #86, "Supporting changes"; Modalities PR #459, commit notes
+ * on mamba2.py); the core then runs on column slices of that row with nothing copied.
+ *
+ * hidden [b][L][d_model] bf16 (row stride hidden_ld); W_in [2HP + 2GN + H][d_model] bf16 and
+ * W_out [d_model][HP] bf16, row-major, 16-byte aligned; the core's parameters and states as for
+ * ssd_mixer_prefill; out [b][L][d_model] bf16 (row stride out_ld). bf16 activations only;
+ * d_model, the strides and 2HP + 2GN + H multiples of 8; the core's shape rules as for
+ * ssd_mixer_prefill. workspace: ssd_mixer_layer_workspace_size bytes, 256-byte aligned; it holds
+ * the packed in_proj output and y, and its status word is read by ssd_mixer_workspace_status.
+ * When the core's norm group is wider than one cluster of the tensor-core kernel (more than 4
+ * heads per group), the norm is finished inside out_proj: the group RMS scale and norm_w are
+ * applied to out_proj's input tiles before their MMAs, so y is not read and written again. */
+SSD_API ssd_status ssd_mixer_layer_prefill(const ssd_dims* dims, int64_t d_model,
+                                           const void* hidden, int64_t hidden_ld,
+                                           const void* W_in, const void* W_out,
+                                           const float* A, const float* D,
+                                           const float* conv_w, const float* conv_b,
+                                           const float* dt_bias, const float* norm_w,
+                                           const float* init_ssm_state, const void* init_conv_state,
+                                           void* out, int64_t out_ld,
+                                           float* final_ssm_state, void* final_conv_state,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream);
+
 /* Bytes of device workspace ssd_mixer_backward needs for `dims`; 0 when the dims are
  * invalid or the shape is one the backward does not run. About (b L (4 HP + Cc + 2 H
  * (P/16) N + H (P/16) + 2 H) + b (L/64) H P N) * 4 bytes: the recompute forward's

@@ -220,3 +220,14 @@ def test_stage_offsets_follow_the_workspace_layout(lib):
     assert off["y_pre"] + b * L * HP * 4 <= sm.ssd_mixer_prefill_workspace_size(d)
     with pytest.raises(sm.SsdError):
         sm.ssd_mixer_prefill_stage_offsets(_dims(headdim=64, dstate=128, nheads=8, ngroups=2))
+
+
+def test_layer_and_projection_refuse_unsupported_arguments(lib):
+    d = _dims(headdim=64, dstate=128, nheads=8, ngroups=2, seqlen=100)
+    assert sm.ssd_mixer_layer_workspace_size(d, 256) > sm.ssd_mixer_prefill_workspace_size(d)
+    assert sm.ssd_mixer_layer_workspace_size(d, 250) == 0                 # d_model not a multiple of 8
+    assert sm.ssd_mixer_layer_workspace_size(_dims(act="f32", headdim=64, dstate=128), 256) == 0
+    # K not a multiple of 8, misaligned workspace: refused before any launch
+    assert lib.ssd_mixer_projection(4, 8, 12, FAKE, 16, FAKE, 16, FAKE, 8, FAKE, None) == sm.SSD_ERR_UNSUPPORTED
+    assert lib.ssd_mixer_projection(4, 8, 16, FAKE, 16, FAKE, 16, FAKE, 8, FAKE + 8, None) == sm.SSD_ERR_INVALID_ARG
+    assert lib.ssd_mixer_projection(0, 8, 16, None, 16, None, 16, None, 8, FAKE, None) == sm.SSD_OK
