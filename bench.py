@@ -49,6 +49,9 @@ HEADLINE = "long_bf16"
 SUB_PREFILL = ("tiny_f32", "small_bf16", "mid_bf16")
 L2_BYTES = 126 * 2**20
 TRAFFIC_FILE = "profiles/dram_traffic_per_launch.json"
+# model width of the layer sub-record: Nemotron-3 Nano, whose Mamba mixer has the mid workload's
+# 64 heads x 64 (Modalities PR #459, commit notes: dimension 2688)
+LAYER_D_MODEL = 2688
 
 
 def parse(argv=None):
@@ -62,10 +65,50 @@ def parse(argv=None):
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="skip the tiny/small/mid prefill sub-records")
+    ap.add_argument("--no-layer", action="store_true", help="skip the whole-layer (projections + core) sub-record")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target length of the CPU sample")
+    ap.add_argument("--profile-case", choices=["long_4k", "layer_mid"], default=None,
+                    help="run one small case for a profiler (3 warm-up calls, then 1) and exit: a long_bf16-shaped "
+                         "prefill of 4096 tokens, or the mid_bf16 layer")
     return ap.parse_args(argv)
+
+
+def profile_case(name: str) -> None:
+    """Three warm-up calls and one more of a case sized for an ncu capture (a few hundred MB on
+    the device, still larger than L2), then exit; prints one line, no benchmark figures."""
+    import torch
+    from hybrid_mamba_ssm_causal_b200 import ssd_mixer as sm
+    from hybrid_mamba_ssm_causal_b200.workloads import WORKLOADS, make_params, round_bf16
+    dev = torch.device("cuda", 0)
+    rng = np.random.default_rng(7)
+    if name == "long_4k":
+        w = WORKLOADS["long_bf16"].with_(seqlen=4096, calls=1)
+    else:
+        w = WORKLOADS["mid_bf16"]
+    d = sm.Dims(w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk, w.dconv, w.eps, w.act)
+    prm = {k: torch.from_numpy(v).float().to(dev) for k, v in make_params(w, rng).items()}
+    bf = lambda *shape: torch.from_numpy(round_bf16(rng.standard_normal(shape, dtype=np.float32))).to(torch.bfloat16).to(dev)
+    HP, GN, H = w.d_inner, w.ngroups * w.dstate, w.nheads
+    if name == "long_4k":
+        x, z, B, C, dt = bf(w.batch, w.seqlen, HP), bf(w.batch, w.seqlen, HP), bf(w.batch, w.seqlen, GN), \
+            bf(w.batch, w.seqlen, GN), bf(w.batch, w.seqlen, H)
+        ws = sm.alloc_workspace(d, dev)
+        run = lambda: sm.prefill(d, x, z, B, C, dt, prm["A"], prm["D"], prm["conv_w"], prm["conv_b"],
+                                 prm["dt_bias"], prm["norm_w"], workspace=ws)
+    else:
+        width = 2 * HP + 2 * GN + H
+        hid = bf(w.batch, w.seqlen, LAYER_D_MODEL)
+        Win = (bf(width, LAYER_D_MODEL).float() / np.sqrt(LAYER_D_MODEL)).to(torch.bfloat16)
+        Wout = (bf(LAYER_D_MODEL, HP).float() / np.sqrt(HP)).to(torch.bfloat16)
+        ws = torch.empty(sm.ssd_mixer_layer_workspace_size(d, LAYER_D_MODEL), dtype=torch.uint8, device=dev)
+        run = lambda: sm.layer_prefill(d, hid, Win, Wout, prm["A"], prm["D"], prm["conv_w"], prm["conv_b"],
+                                       prm["dt_bias"], prm["norm_w"], workspace=ws)
+    for _ in range(4):
+        run()
+    torch.cuda.synchronize()
+    print(f"profile case {name} done", flush=True)
 
 
 def peaks():
@@ -141,6 +184,8 @@ def kernel_bytes(name, w, batch, seqlen, init_states=False) -> int | None:
         return path_bytes(w, batch, seqlen, init_states)
     if name == "tc_norm_finish":       # gated values read and written, partial sums read
         return tok * HP * es * 2 + tok * H * 4 * 4
+    if name == "tc_bc_conv":           # raw B, C read, SiLU(conv) of them written
+        return tok * 2 * GN * es * 2
     return None
 
 
@@ -420,6 +465,9 @@ def main():
     if a.impl == "reference":
         run_reference(a, rank, world)
         return
+    if a.profile_case:
+        profile_case(a.profile_case)
+        return
 
     import torch
     import torch.distributed as dist
@@ -651,6 +699,61 @@ def main():
                 subs[name]["note"] = "fp32 CUDA-core path; latency-bound at this size (no roofline claim)"
             del sets, base, wsp
 
+    # ---------------- the whole mixer layer (in_proj -> core -> out_proj) on the mid workload
+    layer = None
+    if not a.no_layer:
+        from hybrid_mamba_ssm_causal_b200.workloads import make_params, round_bf16
+        wl = WORKLOADS["mid_bf16"]
+        d_model = LAYER_D_MODEL
+        HP, GN, H = wl.d_inner, wl.ngroups * wl.dstate, wl.nheads
+        width = 2 * HP + 2 * GN + H
+        rows = wl.batch * wl.seqlen
+        rng = np.random.default_rng(5)
+        lp = make_params(wl, rng)
+        hid = torch.from_numpy(round_bf16(rng.standard_normal((wl.batch, wl.seqlen, d_model), dtype=np.float32))).to(adt).to(dev)
+        Win = torch.from_numpy(round_bf16((rng.standard_normal((width, d_model), dtype=np.float32) /
+                                           np.float32(np.sqrt(d_model))))).to(adt).to(dev)
+        Wout = torch.from_numpy(round_bf16((rng.standard_normal((d_model, HP), dtype=np.float32) /
+                                            np.float32(np.sqrt(HP))))).to(adt).to(dev)
+        LP = {k: to_dev(lp[k], False, adt) for k in ("A", "D", "conv_w", "conv_b", "dt_bias", "norm_w")}
+        dlay = dims(wl)
+        lws = torch.empty(sm.ssd_mixer_layer_workspace_size(dlay, d_model), dtype=torch.uint8, device=dev)
+        lout = (torch.empty(wl.batch, wl.seqlen, d_model, dtype=adt, device=dev),
+                torch.empty(wl.batch, H, wl.headdim, wl.dstate, device=dev),
+                torch.empty(wl.batch, wl.xbc_channels, 3, dtype=adt, device=dev))
+
+        def lstep(_i):
+            sm.layer_prefill(dlay, hid, Win, Wout, LP["A"], LP["D"], LP["conv_w"], LP["conv_b"], LP["dt_bias"],
+                             LP["norm_w"], None, None, workspace=lws, out=lout)
+
+        lms, llaunch = timed(lstep, max(3, a.steps // 2), max(3, a.warmup))
+        lk = profiled(lib, lstep, max(3, a.steps // 2))
+
+        def lstep_fused(_i):
+            sm.layer_prefill(dlay, hid, Win, Wout, LP["A"], LP["D"], LP["conv_w"], LP["conv_b"], LP["dt_bias"],
+                             LP["norm_w"], None, None, workspace=lws, out=lout, norm_in_out_proj=True)
+
+        lms_fused, _ = timed(lstep_fused, max(3, a.steps // 2), max(3, a.warmup))
+        nrep = max(3, a.steps // 2)
+        fl_in, fl_out = 2.0 * rows * d_model * width, 2.0 * rows * HP * d_model
+        gem = {}
+        gemm_ms = sum(v[0] for k, v in lk.items() if k.startswith("tc_gemm"))
+        if gemm_ms > 0:
+            # two GEMM launches per call: in_proj, then out_proj (with the norm prologue when the
+            # group is wider than a cluster)
+            gem = {"kernel": "tc_gemm (in_proj + out_proj)", "bound": "tensor", "unit": "TFLOP/s",
+                   "achieved": (fl_in + fl_out) * nrep / (gemm_ms * 1e-3) / 1e12,
+                   "peak": tf_burst, "peak_source": peak_src}
+            gem["frac"] = gem["achieved"] / tf_burst
+        layer = {"workload": f"mid_bf16 layer: b{wl.batch} L{wl.seqlen}, d_model {d_model}, in_proj {d_model}->{width}, "
+                             f"core H{H}xP{wl.headdim} G{wl.ngroups} N{wl.dstate}, out_proj {HP}->{d_model}",
+                 "value": job_value(world, rows, lms), "unit": "tokens/s", "ms_per_call": lms,
+                 "ms_per_call_norm_in_out_proj": lms_fused,
+                 "launches_per_call": llaunch / nrep, "gemm_flops_per_call": fl_in + fl_out,
+                 "roofline": gem or None,
+                 "kernels": {k: {"ms_per_call": v[0] / nrep, "launches": v[1]} for k, v in lk.items()}}
+        del hid, Win, Wout, lws, lout
+
     # ---------------- decode workload: 256 sequences, 1000 single-token steps, state in place
     decode_rec = None
     if not a.no_decode:
@@ -736,7 +839,7 @@ def main():
                          "frac": step_bytes / (ms * 1e-3) / 1e9 / hbm, "peak": hbm, "peak_source": peak_src},
             "roofline": roofline, "kernels": {k: {"ms_per_step": v[0] / a.steps, "launches": v[1]}
                                               for k, v in per_kernel.items()},
-            "gpu_launches": launches, "e2e": e2e, "workloads": subs, "decode_workload": decode_rec,
+            "gpu_launches": launches, "e2e": e2e, "workloads": subs, "layer": layer, "decode_workload": decode_rec,
             "backward": bwd, "clocks": ck, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

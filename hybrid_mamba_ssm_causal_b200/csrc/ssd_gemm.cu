@@ -12,9 +12,10 @@
 //   warps 2..5        the epilogue: a TMEM lane (one output row) per thread, 64 columns at a
 //                     time into a 128-byte-swizzled staging tile, stored by TMA (double
 //                     buffered; rows and columns past the matrix are clipped by the store).
-// Optional prologue on A (out_proj of a group norm finished late): every A element of row t
-// and column k is multiplied by row_scale[t][k / scale_group] before its MMA, by the epilogue
-// warps, in shared memory.
+//   warps 6..13       (with a prologue on A only) every A element of row t and column k times
+//                     row_scale[t][k / scale_group] and col_scale[k], in shared memory, before
+//                     its MMAs (out_proj of a group norm finished late); the K-block's column
+//                     scales are staged once in shared memory.
 // All waits are bounded; a wait that gives up sets the status word and stops waiting.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -32,12 +33,13 @@ namespace {
 using namespace tc;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 192, kGemmThreadsScaled = 448;
 constexpr uint32_t kABytes = kBM * kBK * 2, kWBytes = kBN * kBK * 2, kStageBytes = kABytes + kWBytes;
 constexpr uint32_t kOutChunk = 64;                     // columns per staged store
 constexpr uint32_t kOutBytes = kBM * kOutChunk * 2;    // 16 KB
 constexpr uint32_t kOffOut = kStages * kStageBytes;    // 2 staging tiles
-constexpr uint32_t kOffBar = kOffOut + 2 * kOutBytes;
+constexpr uint32_t kOffColScale = kOffOut + 2 * kOutBytes;   // [kStages][64] fp32
+constexpr uint32_t kOffBar = kOffColScale + kStages * kBK * 4;
 // full[4] empty[4] scaled[4] acc_full[2] acc_empty[2]
 constexpr int kNBar = 3 * kStages + 4;
 constexpr uint32_t kOffTmem = kOffBar + kNBar * 8;
@@ -61,7 +63,8 @@ struct GemmArgs {
 __device__ __forceinline__ void gemm_named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 template <bool SCALE>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_tn_kernel(GemmArgs g, const __grid_constant__ GemmMaps maps)
+__global__ void __launch_bounds__(SCALE ? kGemmThreadsScaled : kGemmThreads, 1)
+    gemm_bf16_tn_kernel(GemmArgs g, const __grid_constant__ GemmMaps maps)
 {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -146,44 +149,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_tn_kernel(GemmArgs 
                 mma_commit(acc_full(b));
             }
         }
+    } else if (warp >= 6) {
+        // ------------------------------- A prologue (warps 6..13) -------------------------------
+        if constexpr (SCALE) {
+            const int sid = tid - 192;
+            const int r = sid & 127;            // A row of the tile, and which half of its 8 chunks
+            const int vh = sid >> 7;
+            float* s_cs = reinterpret_cast<float*>(smem + kOffColScale);
+            // every global read is issued well before its use: the column scales one K-block
+            // ahead, the row's group scale one group ahead
+            auto colv = [&](int kcol) { return (sid < kBK && g.col_scale && kcol + sid < g.K) ? g.col_scale[kcol + sid] : 1.0f; };
+            const int ngrp = (g.K + g.scale_group - 1) / g.scale_group;
+            int it = 0;
+            for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+                const int tm = t / tiles_n;
+                const int64_t grow = (int64_t)tm * kBM + r;
+                const float* rs = g.row_scale + grow * g.scale_ld;
+                auto rowv = [&](int grp) { return (grow < g.M && grp < ngrp) ? rs[grp] : 0.0f; };
+                int cur_grp = 0;
+                float cur_sc = rowv(0), next_sc = rowv(1);
+                float ncs = colv(0);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t par = (uint32_t)((it / kStages) & 1);
+                    const int kcol = kb * kBK;
+                    float* cs = s_cs + s * kBK;
+                    if (sid < kBK) cs[sid] = ncs;
+                    if (kb + 1 < nk) ncs = colv(kcol + kBK);
+                    const int grp = kcol / g.scale_group;
+                    if (grp != cur_grp) {
+                        cur_grp = grp;
+                        cur_sc = next_sc;
+                        next_sc = rowv(grp + 1);
+                    }
+                    const float sc = cur_sc;
+                    if (ok && !mbar_wait_bounded(full(s), par, kGemmWait)) ok = false;
+                    gemm_named_sync(2, 256);
+                    unsigned char* a = smem + (size_t)s * kStageBytes;
+#pragma unroll
+                    for (int vv = 0; vv < kBK / 16; ++vv) {   // 16-byte chunk v of row r (128-byte swizzle)
+                        const int v = vh * (kBK / 16) + vv;
+                        uint4* p = reinterpret_cast<uint4*>(a + r * 128 + ((v ^ (r & 7)) << 4));
+                        const float4 c0 = *reinterpret_cast<const float4*>(cs + v * 8);
+                        const float4 c1 = *reinterpret_cast<const float4*>(cs + v * 8 + 4);
+                        float f[8];
+                        unpack_bf16x8(*p, f);
+                        *p = make_uint4(pack_bf16x2(f[0] * sc * c0.x, f[1] * sc * c0.y), pack_bf16x2(f[2] * sc * c0.z, f[3] * sc * c0.w),
+                                        pack_bf16x2(f[4] * sc * c1.x, f[5] * sc * c1.y), pack_bf16x2(f[6] * sc * c1.z, f[7] * sc * c1.w));
+                    }
+                    fence_async_smem();
+                    gemm_named_sync(2, 256);
+                    if (sid == 0) mbar_arrive_local(scaled(s));
+                }
+            }
+        }
     } else {
         // ------------------------------- epilogue (warps 2..5) -------------------------------
         const int q = warp & 3;                 // TMEM lane quadrant this warp may access
         const int row = q * 32 + lane;          // output row within the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const int etid = tid - 64;              // 0..127
-        int it = 0, lt = 0, nst = 0;            // K-blocks scaled, tiles stored, staged chunks issued
+        int lt = 0, nst = 0;                    // tiles stored, staged chunks issued
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
             const int tm = t / tiles_n, tn = t % tiles_n;
-            if constexpr (SCALE) {
-                // the A rows of each K-block times their row's group scale, before the MMAs
-                const int r = etid;             // A row of the tile handled by this thread
-                const int64_t grow = (int64_t)tm * kBM + r;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t par = (uint32_t)((it / kStages) & 1);
-                    if (ok && !mbar_wait_bounded(full(s), par, kGemmWait)) ok = false;
-                    const int kcol = kb * kBK;
-                    const float sc = (grow < g.M) ? g.row_scale[grow * g.scale_ld + kcol / g.scale_group] : 0.0f;
-                    unsigned char* a = smem + (size_t)s * kStageBytes;
-#pragma unroll
-                    for (int v = 0; v < kBK / 8; ++v) {   // 16-byte chunk v of row r (128-byte swizzle)
-                        uint4* p = reinterpret_cast<uint4*>(a + r * 128 + ((v ^ (r & 7)) << 4));
-                        float f[8], cs[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int k = kcol + v * 8 + e;
-                            cs[e] = (g.col_scale && k < g.K) ? g.col_scale[k] : 1.0f;
-                        }
-                        unpack_bf16x8(*p, f);
-                        *p = make_uint4(pack_bf16x2(f[0] * sc * cs[0], f[1] * sc * cs[1]), pack_bf16x2(f[2] * sc * cs[2], f[3] * sc * cs[3]),
-                                        pack_bf16x2(f[4] * sc * cs[4], f[5] * sc * cs[5]), pack_bf16x2(f[6] * sc * cs[6], f[7] * sc * cs[7]));
-                    }
-                    fence_async_smem();
-                    gemm_named_sync(1, 128);
-                    if (etid == 0) mbar_arrive_local(scaled(s));
-                }
-            }
             const int b = lt & 1;
             if (ok && !mbar_wait_bounded(acc_full(b), (uint32_t)((lt >> 1) & 1), kGemmWait)) ok = false;
             fence_after_sync();
@@ -317,7 +345,7 @@ cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int
         cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
         if (e != cudaSuccess) return e;
         LaunchScope ls("tc_gemm_scaled", st);
-        gemm_bf16_tn_kernel<true><<<grid, kGemmThreads, kGemmSmem, st>>>(g, maps);
+        gemm_bf16_tn_kernel<true><<<grid, kGemmThreadsScaled, kGemmSmem, st>>>(g, maps);
     } else {
         cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
         if (e != cudaSuccess) return e;

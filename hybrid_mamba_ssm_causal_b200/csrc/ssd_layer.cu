@@ -6,9 +6,12 @@
 // [z | xBC | dt]; Modalities PR #459, commit notes on mamba2.py, on the packed [z, x, B, C, dt]
 // projection). The core reads x, z, B, C and dt as column slices of that row (its ABI takes a
 // row stride for each), so nothing is copied between the GEMM and the core. When the core's
-// norm group is wider than a thread-block cluster, the core leaves y gated but not normalised;
-// the group RMS scale of every (token, group) and the norm weights are then applied to out_proj's
-// A tiles in shared memory before their MMAs, so y is not read and written a second time.
+// norm group is wider than a thread-block cluster, the norm is finished either by the core's own
+// pass over y (the default), or, on request, inside out_proj: the core leaves y gated but not
+// normalised and the group RMS scale of every (token, group) and the norm weights are applied
+// to out_proj's A tiles in shared memory before their MMAs. The second way saves the pass over y
+// but routes every A tile through shared memory twice more, which costs more than it saves on a
+// B200 at the shapes measured, so it is not the default.
 #include <cuda_bf16.h>
 
 #include "../../include/ssd_mixer.h"
@@ -92,7 +95,7 @@ ssd_status ssd_mixer_layer_prefill(const ssd_dims* d, int64_t d_model, const voi
                                    const float* conv_w, const float* conv_b, const float* dt_bias,
                                    const float* norm_w, const float* init_ssm_state, const void* init_conv_state,
                                    void* out, int64_t out_ld, float* final_ssm_state, void* final_conv_state,
-                                   void* workspace, size_t workspace_bytes, void* stream)
+                                   int norm_in_out_proj, void* workspace, size_t workspace_bytes, void* stream)
 {
     if (!d) return SSD_ERR_INVALID_ARG;
     if (!layer_dims_ok(d, d_model)) return SSD_ERR_UNSUPPORTED;
@@ -125,7 +128,7 @@ ssd_status ssd_mixer_layer_prefill(const ssd_dims* d, int64_t d_model, const voi
     const ssd_status cs = ssd::prefill_call(d, zx + HP, width, zx, width, zx + 2 * HP, width, zx + 2 * HP + GN, width,
                                             zx + 2 * HP + 2 * GN, width, A, D, conv_w, conv_b, dt_bias, norm_w,
                                             init_ssm_state, init_conv_state, y, HP, final_ssm_state, final_conv_state,
-                                            ws + l.core, core_bytes, stream, true, true, &p);
+                                            ws + l.core, core_bytes, stream, norm_in_out_proj != 0, true, &p);
     if (cs != SSD_OK) return cs;
     if (rows == 0) return SSD_OK;
     // out_proj; a norm left to it is applied to its A tiles (group scale and norm weights)

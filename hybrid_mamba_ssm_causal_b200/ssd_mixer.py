@@ -118,7 +118,7 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_layer_workspace_size.argtypes = [ctypes.POINTER(_CDims), I64]
     lib.ssd_mixer_layer_workspace_size.restype = ctypes.c_size_t
     lib.ssd_mixer_layer_prefill.argtypes = ([ctypes.POINTER(_CDims), I64, P, I64, P, P] + [FP] * 6 +
-                                            [FP, P, P, I64, FP, P, P, ctypes.c_size_t, V])
+                                            [FP, P, P, I64, FP, P, ctypes.c_int, P, ctypes.c_size_t, V])
     lib.ssd_mixer_layer_prefill.restype = ctypes.c_int
     lib.ssd_mixer_prefill_path.argtypes = [ctypes.POINTER(_CDims)]
     lib.ssd_mixer_prefill_path.restype = ctypes.c_int
@@ -269,9 +269,11 @@ def ssd_mixer_layer_workspace_size(dims: Dims, d_model: int) -> int:
 
 
 def layer_prefill(dims: Dims, hidden, W_in, W_out, A, D, conv_w, conv_b, dt_bias, norm_w,
-                  init_ssm_state=None, init_conv_state=None, workspace=None, out=None, stream=None):
+                  init_ssm_state=None, init_conv_state=None, workspace=None, out=None, norm_in_out_proj=False,
+                  stream=None):
     """The whole mixer layer (in_proj, the core, out_proj) through ssd_mixer_layer_prefill.
     hidden [b, L, d_model] bf16; W_in [2HP + 2GN + H, d_model]; W_out [d_model, HP].
+    norm_in_out_proj: finish a wide group's norm inside out_proj instead of in the core.
     Returns (out [b, L, d_model], final_ssm_state, final_conv_state)."""
     lib = load_library()
     d_model = hidden.shape[-1]
@@ -296,7 +298,8 @@ def layer_prefill(dims: Dims, hidden, W_in, W_out, A, D, conv_w, conv_b, dt_bias
         ctypes.byref(cd), d_model, ph, hld, _dev(W_in, "W_in"), _dev(W_out, "W_out"), _dev(A, "A"), _dev(D, "D"),
         _dev(conv_w, "conv_w"), _dev(conv_b, "conv_b"), _dev(dt_bias, "dt_bias"), _dev(norm_w, "norm_w"),
         _dev(init_ssm_state, "init_ssm_state"), _dev(init_conv_state, "init_conv_state"), py, yld,
-        _dev(fs, "final_ssm_state"), _dev(fc, "final_conv_state"), _dev(workspace, "workspace"),
+        _dev(fs, "final_ssm_state"), _dev(fc, "final_conv_state"), 1 if norm_in_out_proj else 0,
+        _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "ssd_mixer_layer_prefill")
     return y, fs, fc

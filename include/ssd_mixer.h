@@ -335,9 +335,11 @@ SSD_API size_t ssd_mixer_layer_workspace_size(const ssd_dims* dims, int64_t d_mo
  * d_model, the strides and 2HP + 2GN + H multiples of 8; the core's shape rules as for
  * ssd_mixer_prefill. workspace: ssd_mixer_layer_workspace_size bytes, 256-byte aligned; it holds
  * the packed in_proj output and y, and its status word is read by ssd_mixer_workspace_status.
- * When the core's norm group is wider than one cluster of the tensor-core kernel (more than 4
- * heads per group), the norm is finished inside out_proj: the group RMS scale and norm_w are
- * applied to out_proj's input tiles before their MMAs, so y is not read and written again. */
+ * norm_in_out_proj: when the core's norm group is wider than one cluster of the tensor-core
+ * kernel (more than 4 heads per group), 0 finishes the norm with the core's own pass over y, and
+ * nonzero finishes it inside out_proj instead (the group RMS scale and norm_w applied to
+ * out_proj's input tiles in shared memory before their MMAs; no second pass over y, but more
+ * shared-memory traffic per tile, measured slower on a B200). Ignored for other shapes. */
 SSD_API ssd_status ssd_mixer_layer_prefill(const ssd_dims* dims, int64_t d_model,
                                            const void* hidden, int64_t hidden_ld,
                                            const void* W_in, const void* W_out,
@@ -347,6 +349,7 @@ SSD_API ssd_status ssd_mixer_layer_prefill(const ssd_dims* dims, int64_t d_model
                                            const float* init_ssm_state, const void* init_conv_state,
                                            void* out, int64_t out_ld,
                                            float* final_ssm_state, void* final_conv_state,
+                                           int norm_in_out_proj,
                                            void* workspace, size_t workspace_bytes,
                                            void* stream);
 

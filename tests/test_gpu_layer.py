@@ -8,8 +8,9 @@ to bf16, 2^-9 relative, and the sums run in a different order). The shapes span 
 ssd_mixer_layer_prefill (in_proj -> the core on column slices of the packed [z | x | B | C | dt]
 row -> out_proj) is compared with the fp64 layer oracle (oracle/layer.py) within the bf16
 tolerance 2e-2 on the layer output and both final states, for a norm group held by one cluster
-(4 heads per group: the core normalises) and for a wider group (8 heads per group: out_proj
-applies the group scale and norm weights to its input tiles).
+(4 heads per group: the core normalises) and for a wider group (8 heads per group), with the
+norm finished by the core's own pass or, on request, by out_proj applying the group scale and
+norm weights to its input tiles.
 """
 import numpy as np
 import pytest
@@ -65,15 +66,15 @@ def _layer_case(heads, groups, seqlen, d_model, seed):
     return w, prm, hidden, W_in, W_out, init_ssm, init_conv
 
 
-@pytest.mark.parametrize("heads,groups", [(8, 2), (16, 2)])
-def test_layer_matches_layer_oracle(heads, groups):
+@pytest.mark.parametrize("heads,groups,in_out_proj", [(8, 2, False), (16, 2, False), (16, 2, True)])
+def test_layer_matches_layer_oracle(heads, groups, in_out_proj):
     w, prm, hidden, W_in, W_out, init_ssm, init_conv = _layer_case(heads, groups, 333, 256, seed=61 + heads)
     d = dims_of(w)
     bf = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
     f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).float().cuda()
     P = {k: f32(prm[k]) for k in ("A", "D", "conv_w", "conv_b", "dt_bias", "norm_w")}
     out, fs, fc = sm.layer_prefill(d, bf(hidden), bf(W_in), bf(W_out), P["A"], P["D"], P["conv_w"], P["conv_b"],
-                                   P["dt_bias"], P["norm_w"], f32(init_ssm), bf(init_conv))
+                                   P["dt_bias"], P["norm_w"], f32(init_ssm), bf(init_conv), norm_in_out_proj=in_out_proj)
     torch.cuda.synchronize()
     ref_out, ref_fs, ref_fc = oracle_layer(oracle_dims(d), hidden, W_in.T, W_out.T, prm["A"], prm["D"], prm["conv_w"],
                                            prm["conv_b"], prm["dt_bias"], prm["norm_w"], init_ssm, init_conv)
