@@ -18,7 +18,7 @@ WorkspaceLayout prefill_workspace_layout(int64_t b, int64_t L, int64_t rows, int
         w.status = 0;
         w.xbc = w.delta = w.lam = w.states = w.ypre = 256;
         w.bcp = 256;
-        size_t off = align256(256 + (size_t)rows * (size_t)(2 * G * N) * 2);
+        size_t off = align256(256 + prefill_bc_blocks(b, rows) * (size_t)(2 * G * N) * kBcBlockTokens * 2);
         w.ssp = off;
         if (prefill_tc_split(H, G)) off = align256(off + (size_t)(rows * H) * (size_t)prefill_ws_partials_per_head() * 4);
         w.total = off;

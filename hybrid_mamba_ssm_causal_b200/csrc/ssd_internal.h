@@ -54,7 +54,8 @@ struct PrefillParams {
     float* states;   // [b][nc][H][P][N] chunk states, then states entering each chunk
     float* ypre;     // [b][L][HP] y before the gate and norm
     float* ssp;      // tensor-core path, groups wider than one cluster: [rows][H][parts] sums of g^2
-    void* bcp;       // tensor-core path: [rows][2 GN] bf16, SiLU(conv) of the B and C channels
+    void* bcp;       // tensor-core path: SiLU(conv) of the B and C channels, bf16, blocked (see
+                     // prefill_bc_blocks)
     // Packed variable-length sequences on state slots (cu_seqlens != nullptr): b sequences,
     // L = total packed tokens, sequence i owns rows cu_seqlens[i] .. cu_seqlens[i+1]-1; its
     // states are the slot slot_idx[i] (identity when null) of init_ssm/init_conv, which
@@ -158,6 +159,13 @@ cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int
 // The state-only pass on the tensor-core path: final states and decay, no output rows.
 cudaError_t launch_prefill_state_ws(const PrefillParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream);
+// The tensor-core path keeps SiLU(conv) of B and C in the workspace as 32 KB chunks, one per
+// (128-token block of a sequence, matrix B or C, group): chunk ((s + floor(start_s / 128) + k) * 2
+// + matrix) * G + group holds block k of sequence s (first packed row start_s) in the MMA operand
+// layout [16 vectors of 8 channels][128 tokens][8]. Sequences never share a chunk, and
+// prefill_bc_blocks(b, rows) = b + rows / 128 + 1 bounds the block index.
+constexpr int64_t kBcBlockTokens = 128;
+inline size_t prefill_bc_blocks(int64_t b, int64_t rows) { return (size_t)(b + rows / kBcBlockTokens + 1); }
 int prefill_ws_partials_per_head();
 
 // H_in(r) of a sequence split into pieces: init (NULL = zeros) carried through pieces 0..r-1.

@@ -12,44 +12,52 @@
 //
 // Two kernels per call (three when the norm group is wider than a cluster):
 //   bc_conv       SiLU(conv) of the B and C channels, once for all heads of a group (every
-//                 head reads the same B', C'), into the workspace as [token][2*G*N] bf16;
+//                 head reads the same B', C'), into the workspace as one 32 KB chunk per
+//                 (128-token block, matrix, group), already in the MMA operand layout;
 //   ssd_prefill_ws_kernel  one CTA per (sequence, head): the x conv, the scan, the chunked SSD
 //                 on tensor cores, the D skip and the gated norm. When a thread-block cluster
 //                 holds the whole group (2 or 4 heads), the norm's per-token sums of squares go
 //                 to every peer with st.async; wider groups write gated values and partial sums
 //                 and a light pass finishes the norm.
 //
-// Data movement: the raw x rows of a block (with the 3-token conv halo) and the block's B', C'
-// arrive by TMA (B'/C' land directly in the MMA operand layout); z is read straight into
-// registers (64 contiguous bytes per consumer thread, issued a few thousand cycles before
-// use); y leaves through a TMA store of a 128-byte-swizzled tile; the decay-masked M goes from
-// registers into TMEM and feeds M x' as the TMEM A operand.
+// Data movement: the raw x rows of a block (with the 3-token conv halo) arrive by TMA as one
+// 128-byte-swizzled box, double-buffered; the block's B', C' by two contiguous bulk copies; z is
+// brought into L2 by a TMA prefetch a block ahead and read into registers (64 contiguous bytes
+// per consumer thread) during the state update; y leaves through a TMA store of a
+// 128-byte-swizzled tile; the decay-masked M goes from registers into TMEM and feeds M x' as the
+// TMEM A operand. Every copy moves rows of at least 128 bytes: the copy engine of an SM handles
+// requests at a limited rate, and 16-byte pieces (8 channels) left it the slowest stage.
 //
 // Roles (512 threads). A tcgen05.mma issue holds its thread about as long as the MMAs take,
-// so one thread that does nothing else issues them all:
+// so one thread that does nothing else issues them all, in the order the consumer needs them:
+// M x' of block k-1, then C'B'^T of block k (so the consumer's M of block k never waits for the
+// state-dependent products), then C'H^T and B'^T(x'w) of block k:
 //   producer warps 0..6  : the softplus + cumsum (warps 3..6) and the conv + SiLU of x' and
 //                          x'w of block k+1 while the MMAs of block k run;
-//   control warp 7       : (one lane) the TMA of B'/C', the MMAs C'B'^T, C'H^T, B'^T(x'w) of
-//                          block k once its operands are in, and M x' once the consumer has
-//                          written M;
-//   consumer warps 8..15 : for block k: the masked decay product M, the state update, the
-//                          group norm of block k-1, then the epilogue of block k.
+//   control warp 7       : (one lane) the copies of B'/C', M x' of block k-1 once the consumer
+//                          has written M, C'B'^T of block k once B', C' are in, C'H^T and
+//                          B'^T(x'w) of block k once x'w and H^T are in;
+//   consumer warps 8..15 : for block k: the masked decay product M (then M x' may start), the
+//                          state update while M x' runs, the group norm of block k-1, then the
+//                          epilogue of block k.
 // Variants: packed variable-length sequences on state slots (a CTA reads its sequence's
 // rows, length and slot from device arrays), and STATE_ONLY (final states and decay only).
 // Hand-offs use mbarriers (all waits bounded):
-//   bar0   MMA1-3 of a block done (tensor-core commit)     bar1  MMA4 done
-//   barBC  B' and C' of a block have landed (TMA)
+//   barCB  C'B'^T of a block done     bar0  C'H^T and B'^T(x'w) done     bar1  M x' done
+//   (tensor-core commits)
+//   barBC  B' and C' of a block have landed (bulk copies)
 //   barP   producer: block k's x', x'w and cumsum are in shared memory (3 slots: the producer
 //          may arrive for blocks k+1 and k+2 before a slow consumer waits for k)
-//   barC   consumer: C'B'^T and S^T of block k read from TMEM, M of block k written to TMEM,
-//          H^T of block k+1 written to shared memory
+//   barM   consumer (one arrival per warp): C'B'^T of block k read, M of block k in TMEM
+//   barH   consumer (one arrival per warp): S^T of block k read, H^T of block k+1 written to
+//          shared memory, so the MMAs of block k+1 may start
 //   barE2  consumer: a block's x' and cumsum slots are free again (3 slots: x' and the cumsum
 //          live until the epilogue, so they rotate through three buffers)
 //   barW   the MMAs of a block are done, so its x'w slot is free again (2 slots: x'w is read
 //          only by the MMA B'^T(x'w), so two buffers suffice)
 //   barN3  the sums of squares of a block from every CTA of the cluster have landed
 //          (st.async transaction bytes; 3 slots)
-//   barTX  TMA of the raw x rows
+//   barTX  TMA of the raw x rows (one per stage)
 // Barriers waited two blocks back use two slots, so a waiter never meets a barrier that
 // has moved two phases past the one it expects. The group norm of block k is finished one
 // block late (its gated values wait in TMEM); a peer can be at most two blocks ahead of
@@ -80,11 +88,13 @@ constexpr int kThreads = 512;
 constexpr int kProd = 224;    // producer threads (warps 0..6)
 constexpr int kCtl = 224;     // the control thread (warp 7, lane 0)
 constexpr int kCons = 256;    // first consumer thread (warps 8..15)
+constexpr int kConsWarps = (kThreads - kCons) / 32;
 constexpr int kScan0 = 96;    // the cumsum runs on producer threads 96..223 (warps 3..6)
-// Raw staging of the head's 8-channel x vectors: tokens t0-8 .. t0+127 of a block, so rows
-// 5..7 hold the conv halo and rows 8..135 the block's tokens; 2176 bytes per vector, a
-// multiple of 128. One TMA box fills all 8 vectors.
-constexpr int kStageRows = 136, kStageTok = 8, kVX = kP / 8;
+// Raw staging of the head's x channels: tokens t0-3 .. t0+127 of a block, so rows 0..2 hold the
+// conv halo and rows 3..130 the block's tokens; one TMA box of 131 rows of 128 bytes, 128-byte
+// swizzled (16-byte piece v of row r at piece v ^ (r % 8)), 1024-byte aligned.
+constexpr int kStageRows = 131, kStageTok = 3, kVX = kP / 8;
+__device__ __forceinline__ int stage_u4(int r, int v) { return r * 8 + (v ^ (r & 7)); }
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
 
@@ -105,14 +115,19 @@ struct WsLayout {
     static constexpr uint32_t OFF_C = 0, OFF_B = 32768, OFF_Y = 65536, OFF_X = 81920,
                               OFF_XW = OFF_X + 3 * 16384, OFF_H = OFF_XW + 2 * 16384, OFF_STAGE = OFF_H + 16384;
     static constexpr uint32_t STAGE_BYTES = (uint32_t)kStageRows * kP * 2;
-    static constexpr uint32_t OFF_MISC = OFF_STAGE + ((STAGE_BYTES + 127) / 128) * 128;
-    // fp32 arrays: lam, delta, v (3 slots each), scan scratch, sums of squares [3][R][2][128],
-    // conv taps and biases of the head's x channels, norm weights
-    static constexpr uint32_t F_LAM = 0, F_DL = 384, F_V = 768, F_SCAN = 1152, F_RED = 1168,
+    static constexpr uint32_t STAGE_PITCH = ((STAGE_BYTES + 1023) / 1024) * 1024;   // swizzle atoms
+    // two raw x stages (the rows of block k+1 arrive while block k is convolved) where shared
+    // memory allows; one for clusters of 4, whose exchange buffer for the norm sums is larger
+    static constexpr int XBUF = R <= 2 ? 2 : 1;
+    static_assert(OFF_STAGE % 1024 == 0, "the swizzled x stage needs 1024-byte alignment");
+    static constexpr uint32_t OFF_MISC = OFF_STAGE + XBUF * STAGE_PITCH;
+    // fp32 arrays: lam, delta, v, the segment factors g (3 slots each), scan scratch, sums of
+    // squares [3][R][2][128], conv taps and biases of the head's x channels, norm weights
+    static constexpr uint32_t F_LAM = 0, F_DL = 384, F_V = 768, F_G = 1152, F_SCAN = 1536, F_RED = 1552,
                               F_CW = F_RED + 3 * R * 2 * 128, F_CB = F_CW + kP * 4, F_NW = F_CB + kP,
                               F_END = F_NW + kP;
     static constexpr uint32_t OFF_BAR = OFF_MISC + ((F_END * 4 + 15) / 16) * 16;
-    static constexpr int NBAR = 16;  // bar0 bar1 barBC barP[3] barC barE2[3] barW[2] barN3[3] barTX
+    static constexpr int NBAR = 19;  // bar0 bar1 barBC barP[3] barM barE2[3] barW[2] barN3[3] barTX[2] barH barCB
     static constexpr uint32_t OFF_TSLOT = OFF_BAR + NBAR * 8;
     static constexpr uint32_t TOTAL = OFF_TSLOT + 16;
     static_assert(TOTAL <= 232448, "dynamic shared memory above the 227 KB a CTA may use");
@@ -197,8 +212,9 @@ __device__ __forceinline__ SeqOf seq_of(const PrefillParams& p, int64_t t)
 // SiLU(conv) of the B and C channels (the first nch of the 2*G*N), once per token for all the
 // heads that read them. One thread per (8-channel vector, run of kBcRun tokens): its taps in
 // registers and the run's kBcRun + 3 raw rows loaded at once; before a sequence's first token
-// the window reads its initial conv state (zeros without one). Output [token][2*G*N] bf16 in
-// the workspace.
+// the window reads its initial conv state (zeros without one). Output in the workspace as one
+// 32 KB chunk per (128-token block of a sequence, matrix, group) in the MMA operand layout
+// (prefill_bc_blocks), so the main kernel fetches each with one contiguous copy.
 constexpr int kBcRun = 4;
 __global__ void __launch_bounds__(256, 2) bc_conv_kernel(PrefillParams p, int nch)
 {
@@ -208,6 +224,7 @@ __global__ void __launch_bounds__(256, 2) bc_conv_kernel(PrefillParams p, int nc
     if (v * 8 >= nch || t0 >= rows) return;
     const int64_t c0 = v * 8;                       // channel within [B | C]
     const bool isC = c0 >= GN;
+    const int64_t cg = (isC ? c0 - GN : c0) / kN, cv = ((isC ? c0 - GN : c0) % kN) / 8;   // group, vector
     const __nv_bfloat16* src = (const __nv_bfloat16*)(isC ? p.C : p.B) + (isC ? c0 - GN : c0);
     const int64_t ld = isC ? p.C_ld : p.B_ld;
     float w[8][4], bb[8];
@@ -253,16 +270,24 @@ __global__ void __launch_bounds__(256, 2) bc_conv_kernel(PrefillParams p, int nc
         float o[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) o[e] = tc::silu_fast(acc[e]);
-        store_vec<__nv_bfloat16>((__nv_bfloat16*)p.bcp + t * 2 * GN + c0, o);
+        // block k of sequence s, row pos of this vector's [128 tokens][8] slab of the chunk
+        const int64_t pos = t - sq.start;
+        __nv_bfloat16* slab = (__nv_bfloat16*)p.bcp +
+                              ((((sq.s + sq.start / kT + pos / kT) * 2 + (isC ? 1 : 0)) * p.G + cg) * (kN / 8) + cv) * (kT * 8);
+        store_vec<__nv_bfloat16>(slab + (pos % kT) * 8, o);
+        // the rows of a sequence's last block past its end are zeros (the MMAs read the whole block)
+        if (pos == sq.len - 1) {
+            for (int64_t r = pos % kT + 1; r < kT; ++r)
+                *reinterpret_cast<uint4*>(slab + r * 8) = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
 }
 
-// Tensor maps of x viewed as [b][vector][token][8 channels] (bf16; a vector is 8 consecutive
-// channels), boxes of 136 tokens x the head's 8 vectors; of B', C' (the workspace) the same
-// way, boxes of 128 tokens x 16 vectors (a group's N channels); of y as [b][L][channels],
-// boxes of 64 channels x 128 tokens with 128-byte swizzling.
+// Tensor maps of x, y and z as [b][L][channels] (bf16), boxes of one head's 64 channels (128
+// bytes) with 128-byte swizzling: 131 tokens for x (a block and its conv halo), 128 for y and z
+// (z only to prefetch a block into L2 a block ahead of the epilogue that reads it).
 struct WsMaps {
-    CUtensorMap x, bc, y;
+    CUtensorMap x, y, z;
 };
 
 // STATE_ONLY: the state-only pass (final states and decay of a prefill, no output rows): the
@@ -298,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     float* s_lam = mf + Lo::F_LAM;
     float* s_dl = mf + Lo::F_DL;
     float* s_v = mf + Lo::F_V;
+    float* s_g = mf + Lo::F_G;
     float* s_scan = mf + Lo::F_SCAN;
     float* s_red = mf + Lo::F_RED;     // [3 slots][R CTAs][2 halves][128 rows]
     float* s_cw = mf + Lo::F_CW;
@@ -311,9 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const uint32_t aC = s_base + Lo::OFF_C, aB = s_base + Lo::OFF_B;
     const uint32_t aX = s_base + Lo::OFF_X, aXW = s_base + Lo::OFF_XW, aH = s_base + Lo::OFF_H;
     const uint32_t bar0 = smem_u32(&bars[0]), bar1 = smem_u32(&bars[1]), barBC = smem_u32(&bars[2]);
-    const uint32_t barP = smem_u32(&bars[3]), barC = smem_u32(&bars[6]);
+    const uint32_t barP = smem_u32(&bars[3]), barM = smem_u32(&bars[6]);
     const uint32_t barE2 = smem_u32(&bars[7]), barW = smem_u32(&bars[10]), barN3 = smem_u32(&bars[12]);
-    const uint32_t barTX = smem_u32(&bars[15]);
+    const uint32_t barTX = smem_u32(&bars[15]), barH = smem_u32(&bars[17]), barCB = smem_u32(&bars[18]);
+    constexpr int XBUF = Lo::XBUF;
+    constexpr int kStageU4 = (int)(Lo::STAGE_PITCH / 16);   // one raw x stage, in 16-byte units
     // ring slots of block k: x', the cumsum and barP/barE2 rotate by 3, x'w and barW by 2
     auto s3 = [](int64_t k) { return (uint32_t)(k % 3); };
     auto p3 = [](int64_t k) { return (uint32_t)((k / 3) & 1); };
@@ -334,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     }
     if (!STATE_ONLY && tid < kP) s_nw[tid] = p.norm_w[(int64_t)h * kP + tid];
     if (tid == 0) {
-        for (int i = 0; i < Lo::NBAR; ++i) mbar_init(smem_u32(&bars[i]), 1);
+        for (int i = 0; i < Lo::NBAR; ++i) mbar_init(smem_u32(&bars[i]), (i == 6 || i == 17) ? kConsWarps : 1);
         fence_mbar_init();
         prefetch_tmap(&maps.x);
-        prefetch_tmap(&maps.bc);
+        if (!STATE_ONLY) prefetch_tmap(&maps.z);
     }
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
 
@@ -370,44 +398,56 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     bool ok = true;
 
     const int64_t nblk = (seqlen + kT - 1) / kT;
-    const __nv_bfloat16* gdt = (const __nv_bfloat16*)p.dt;
     auto blen = [&](int64_t k) { return (int)min((int64_t)kT, seqlen - k * kT); };
 
     if (tid < kProd) {
         // =========================== producer (warps 0..6) ===========================
-        // raw x rows t0-8 .. t0+127 of block kb (TMA, one box of the head's 8 vectors); rows
-        // outside the sequence read as zeros
+        // raw x rows t0-8 .. t0+127 of block kb (TMA, one box of the head's 8 vectors) into stage
+        // kb % XBUF; rows outside the sequence read as zeros
         auto load_x = [&](int64_t kb) {
-            mbar_arrive_expect_tx(barTX, (uint32_t)kVX * kStageRows * 16);
-            tma_load_4d(smem_u32(stage), &maps.x, 0, tmap_t0 + (int)(kb * kT) - kStageTok, h * kVX, tmap_b, barTX);
+            const uint32_t bx = barTX + 8 * (uint32_t)(kb % XBUF);
+            mbar_arrive_expect_tx(bx, Lo::STAGE_BYTES);
+            tma_load_3d(smem_u32(stage + (kb % XBUF) * kStageU4), &maps.x, h * kP, tmap_t0 + (int)(kb * kT) - kStageTok,
+                        tmap_b, bx);
+        };
+        auto wait_x = [&](int64_t kb) {
+            return mbar_wait_bounded(barTX + 8 * (uint32_t)(kb % XBUF), (uint32_t)((kb / XBUF) & 1), kWaitLimit);
         };
         // softplus and cumsum of block kb into its slot (threads kScan0.., token tid - kScan0),
         // then dt of block kb + 1, a whole block ahead of its use
-        float dt_next = 0.0f;
+        // raw bf16 bits of the next block's dt, widened only when used, so the load's latency is
+        // not waited for until a block later
+        uint32_t dt_next = 0u;
+        const unsigned short* gdt16 = reinterpret_cast<const unsigned short*>(p.dt);
         const int tok = tid - kScan0;
         auto scan_block = [&](int64_t kb) {
             const int slb = (int)s3(kb);
             float dl = 0.0f, a2 = 0.0f;
             if (tok < blen(kb)) {
-                dl = softplus(dt_next + bias);
+                dl = softplus(__uint_as_float(dt_next << 16) + bias);
                 a2 = dl * A2;
             }
             if (kb + 1 < nblk && (kb + 1) * kT + tok < seqlen)
-                dt_next = __bfloat162float(gdt[(row0 + (kb + 1) * kT + tok) * p.dt_ld + h]);
+                dt_next = gdt16[(row0 + (kb + 1) * kT + tok) * p.dt_ld + h];
             const float lam = scan128(a2, s_scan);
             s_lam[slb * kT + tok] = lam;
             s_dl[slb * kT + tok] = dl;
             // exp2(lam_i - lam_j) = exp2(lam_i) * exp2(-lam_j) while every factor stays a
             // normal fp32 number (rows with lam_i > -96); chosen per row from its past only
             s_v[slb * kT + tok] = (lam > -96.0f) ? ex2(-lam) * dl : 0.0f;
+            // for rows past that range: exp2(lam_i - lam_j) = exp2(lam_i - lam_s) * exp2(lam_s - lam_j)
+            // with s the first token of j's 8-token segment; g_j = exp2(lam_s - lam_j) * delta_j
+            const float lam_s = __shfl_sync(0xffffffffu, lam, (tid & 31) & ~7);
+            s_g[slb * kT + tok] = ex2(lam_s - lam) * dl;
         };
-        // conv + SiLU of the head's 8 staged x vectors of block kb into x' and x'w. TPV threads
-        // per vector, each taking rows i = t % TPV + TPV m, two at a time, so a warp reads
-        // consecutive staged rows and writes consecutive canonical rows (conflict-free); a
-        // thread keeps its taps in registers.
+        // conv + SiLU of the head's 8 staged x vectors of block kb into x' and x'w. Thread t takes
+        // vector t / TPV and run t % TPV of its 128 tokens (4 or 5 consecutive tokens), sliding a
+        // window of three widened raw rows along the run, so each raw row is read and widened
+        // about 1.7 times instead of once per tap. A quarter warp covers 8 runs of one vector:
+        // its staged rows (131-row pitch) and its x' rows fall in distinct shared-memory banks.
         auto conv_x = [&](int64_t kb) {
             constexpr int TPV = kProd / kVX;
-            static_assert(kProd % kVX == 0, "conv work split");
+            static_assert(kProd % kVX == 0 && 4 * TPV <= kT && kT <= 5 * TPV, "runs of 4 or 5 tokens");
             const int len = blen(kb);
             const int slb = (int)s3(kb);
             const float* lamb = s_lam + slb * kT;
@@ -415,8 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             const float lam_end = lamb[kT - 1];
             unsigned char* sX = smem + Lo::OFF_X + slb * 16384;
             unsigned char* sXW = smem + Lo::OFF_XW + (uint32_t)(kb & 1) * 16384;
-            const int v = tid / TPV;
+            const int v = tid / TPV, run = tid % TPV;
+            const int r0 = (kT * run) / TPV, r1 = (kT * (run + 1)) / TPV;
             const int c0 = v * 8;
+            // staged rows of tokens r0-3 .. r0+4 (the last only for runs of five)
+            const uint4* stg = stage + (kb % XBUF) * kStageU4;
+            const int rr0 = kStageTok - 3 + r0;
             float2 wr[4][4], br[4];
             {
                 const float2* cw2 = reinterpret_cast<const float2*>(s_cw) + (c0 / 2) * 4;
@@ -428,69 +472,79 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     for (int kk = 0; kk < 4; ++kk) wr[j][kk] = cw2[j * 4 + kk];
                 }
             }
-#pragma unroll 1
-            for (int i0 = tid % TPV; i0 < kT; i0 += 2 * TPV) {
-                const bool two = i0 + TPV < kT;
-                uint4 raw[2][4];
+            float2 win[3][4];   // widened raw rows of tokens i-3, i-2, i-1 (channel pairs)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) raw[0][kk] = stage[v * kStageRows + kStageTok - 3 + i0 + kk];
-                if (two) {
+            for (int e = 0; e < 3; ++e) {
+                const uint4 r = stg[stage_u4(rr0 + e, v)];
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) raw[1][kk] = stage[v * kStageRows + kStageTok - 3 + i0 + TPV + kk];
+                for (int j = 0; j < 4; ++j) win[e][j] = bf2_to_f2((&r.x)[j]);
+            }
+#pragma unroll
+            for (int st = 0; st < 5; ++st) {
+                const int i = r0 + st;
+                if (st == 4 && i >= r1) break;
+                float2 cur[4];
+                {
+                    const uint4 r = stg[stage_u4(rr0 + 3 + st, v)];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) cur[j] = bf2_to_f2((&r.x)[j]);
                 }
+                float2 o[4];
+                if (i < len) {
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (u == 1 && !two) break;
-                    const int i = i0 + u * TPV;
-                    float2 o[4];
-                    if (i < len) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {   // channel pair (c0 + 2j, c0 + 2j + 1)
-                            float2 vv = fma2(wr[j][0], bf2_to_f2((&raw[u][0].x)[j]), br[j]);
-                            vv = fma2(wr[j][1], bf2_to_f2((&raw[u][1].x)[j]), vv);
-                            vv = fma2(wr[j][2], bf2_to_f2((&raw[u][2].x)[j]), vv);
-                            vv = fma2(wr[j][3], bf2_to_f2((&raw[u][3].x)[j]), vv);
-                            o[j] = silu2(vv);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) o[j] = make_float2(0.0f, 0.0f);
+                    for (int j = 0; j < 4; ++j) {   // channel pair (c0 + 2j, c0 + 2j + 1)
+                        float2 vv = fma2(wr[j][0], win[0][j], br[j]);
+                        vv = fma2(wr[j][1], win[1][j], vv);
+                        vv = fma2(wr[j][2], win[2][j], vv);
+                        vv = fma2(wr[j][3], cur[j], vv);
+                        o[j] = silu2(vv);
                     }
-                    const float2 wgt = splat2((i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f);
-                    const uint4 u8 = make_uint4(pack_f2(o[0]), pack_f2(o[1]), pack_f2(o[2]), pack_f2(o[3]));
-                    const uint4 uw = make_uint4(pack_f2(mul2(o[0], wgt)), pack_f2(mul2(o[1], wgt)),
-                                                pack_f2(mul2(o[2], wgt)), pack_f2(mul2(o[3], wgt)));
-                    *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
-                    *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) o[j] = make_float2(0.0f, 0.0f);
+                }
+                const float2 wgt = splat2((i < len) ? ex2(lam_end - lamb[i]) * dlb[i] : 0.0f);
+                const uint4 u8 = make_uint4(pack_f2(o[0]), pack_f2(o[1]), pack_f2(o[2]), pack_f2(o[3]));
+                const uint4 uw = make_uint4(pack_f2(mul2(o[0], wgt)), pack_f2(mul2(o[1], wgt)),
+                                            pack_f2(mul2(o[2], wgt)), pack_f2(mul2(o[3], wgt)));
+                *reinterpret_cast<uint4*>(sX + canon_off(i, c0, kP)) = u8;
+                *reinterpret_cast<uint4*>(sXW + canon_off(i, c0, kP)) = uw;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    win[0][j] = win[1][j];
+                    win[1][j] = win[2][j];
+                    win[2][j] = cur[j];
                 }
             }
         };
         if (nblk > 0) {
-            if (tid == 0) load_x(0);
+            if (tid == 0) {
+                for (int64_t kb = 0; kb < XBUF && kb < nblk; ++kb) load_x(kb);
+            }
             if (tid >= kScan0) {
-                if (tok < seqlen) dt_next = __bfloat162float(gdt[(row0 + tok) * p.dt_ld + h]);
+                if (tok < seqlen) dt_next = gdt16[(row0 + tok) * p.dt_ld + h];
                 scan_block(0);
             }
         }
         // the three rows before the sequence hold the initial conv state (zeros without one), not
         // the TMA's fill or a neighbouring packed sequence: written once block 0's rows have landed
         if (nblk == 0 || init_conv || varlen) {
-            if (nblk > 0 && ok && !mbar_wait_bounded(barTX, 0, kWaitLimit)) ok = false;
+            if (nblk > 0 && ok && !wait_x(0)) ok = false;
             for (int e = tid; e < 3 * kP; e += kProd) {
                 const int kk = e / kP, c = e % kP;
                 __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
                 if (init_conv) v = ((const __nv_bfloat16*)p.init_conv)[(sidx * Cc + (int64_t)h * kP + c) * 3 + kk];
-                reinterpret_cast<__nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + kk)[c % 8] = v;
+                reinterpret_cast<__nv_bfloat16*>(stage + stage_u4(kStageTok - 3 + kk, c / 8))[c % 8] = v;
             }
         }
         // x' and x'w of block 0 (the cumsum of block 0 is in its slot)
         if (nblk > 0) {
-            if (ok && !mbar_wait_bounded(barTX, 0, kWaitLimit)) ok = false;
+            if (ok && !wait_x(0)) ok = false;
             named_sync(kBarProd, kProd);
             conv_x(0);
             fence_async_smem();
             named_sync(kBarProd, kProd);
-            if (tid == 32 && nblk > 1) load_x(1);   // the raw x rows have been read
+            if (tid == 32 && XBUF < nblk) load_x(XBUF);   // stage 0 has been read
             if (tid == 0) mbar_arrive_local(barP);
         }
         // while the MMAs of earlier blocks run: the cumsum, x' and x'w of block m, into the x' and
@@ -508,12 +562,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 if (m >= 2 && ok && !mbar_wait_bounded(barW + 8 * (uint32_t)(m & 1), (uint32_t)(((m - 2) >> 1) & 1), kWaitLimit))
                     ok = false;
             }
-            if (ok && !mbar_wait_bounded(barTX, (uint32_t)(m & 1), kWaitLimit)) ok = false;
+            if (ok && !wait_x(m)) ok = false;
             named_sync(kBarProd, kProd);
             conv_x(m);
             fence_async_smem();
             named_sync(kBarProd, kProd);
-            if (tid == 32 && m + 1 < nblk) load_x(m + 1);
+            if (tid == 32 && m + XBUF < nblk) load_x(m + XBUF);   // its stage has been read
             if (tid == 0) mbar_arrive_local(barP + 8 * s3(m));
         }
         // final conv state of the head's x channels: the last three raw inputs
@@ -521,8 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         named_sync(kBarProd, kProd);
         for (int e = tid; e < 3 * kP; e += kProd) {
             const int kk = e / kP, c = e % kP;
+            const uint4* stl = stage + (nblk > 0 ? ((nblk - 1) % XBUF) * kStageU4 : 0);
             const __nv_bfloat16 v =
-                reinterpret_cast<const __nv_bfloat16*>(stage + (c / 8) * kStageRows + kStageTok - 3 + len_last + kk)[c % 8];
+                reinterpret_cast<const __nv_bfloat16*>(stl + stage_u4(kStageTok - 3 + len_last + kk, c / 8))[c % 8];
             ((__nv_bfloat16*)p.final_conv)[(sidx * Cc + (int64_t)h * kP + c) * 3 + kk] = v;
         }
         // the group's first head also writes the B/C part: the last three raw inputs (with the
@@ -558,28 +613,50 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             const uint32_t id_yi = idesc_bf16(128, 64, 0, 1);
             // B' (and C') of block kb: [16 vectors][128 tokens][8] each, straight into the operand
             // layout; tokens past the end of the call read as zeros
+            // (the B/C pass wrote each as one contiguous chunk of the workspace; rows past the
+            // sequence's end are zeros there)
             auto load_bc = [&](int64_t kb) {
-                mbar_arrive_expect_tx(barBC, (STATE_ONLY ? 1u : 2u) * (uint32_t)kT * kN * 2);
-                const int t0 = tmap_t0 + (int)(kb * kT);
-                tma_load_4d(aB, &maps.bc, 0, t0, g * (kN / 8), tmap_b, barBC);
-                if (!STATE_ONLY) tma_load_4d(aC, &maps.bc, 0, t0, (int)(GN / 8) + g * (kN / 8), tmap_b, barBC);
+                constexpr uint32_t kChunk = (uint32_t)kT * kN * 2;
+                mbar_arrive_expect_tx(barBC, (STATE_ONLY ? 1u : 2u) * kChunk);
+                const unsigned char* cB =
+                    (const unsigned char*)p.bcp + (((bi + row0 / kT + kb) * 2) * p.G + g) * (int64_t)kChunk;
+                bulk_load(aB, cB, kChunk, barBC);
+                if (!STATE_ONLY) bulk_load(aC, cB + (int64_t)p.G * kChunk, kChunk, barBC);
             };
             if (nblk > 0) load_bc(0);
+            // M x' of block kb, once every consumer warp has written its rows of M
+            auto mma_yi = [&](int64_t kb) {
+                if (ok && !mbar_wait_bounded(barM, (uint32_t)(kb & 1), kWaitLimit)) ok = false;
+                fence_after_sync();
+                const uint32_t aXs = aX + 16384 * s3(kb);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + kColYi, tmem + kColM + kk * 8, sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
+                mma_commit(bar1);
+            };
             for (int64_t k = 0; k < nblk; ++k) {
                 const int sl = (int)(k & 1);
                 const uint32_t par = (uint32_t)(k & 1);
-                // this block's x' and x'w (barP), B' and C' (barBC); the consumer has read C'B'^T
-                // and S^T of block k-1 and written H^T for this block (barC)
+                if constexpr (!STATE_ONLY) {
+                    if (k >= 1) mma_yi(k - 1);   // also: C'B'^T of block k-1 has been read
+                    // C'B'^T of this block as soon as its B' and C' are in
+                    if (ok && !mbar_wait_bounded(barBC, par, kWaitLimit)) ok = false;
+                    fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tmem + kColCB, sdesc(aC + kk * 4096, 2048, 128), sdesc(aB + kk * 4096, 2048, 128), id_cb, kk > 0);
+                    mma_commit(barCB);
+                } else {
+                    if (ok && !mbar_wait_bounded(barBC, par, kWaitLimit)) ok = false;
+                }
+                // this block's x'w (barP); the consumer has read S^T of block k-1 and written H^T
+                // for this block (barH)
                 if (ok && !mbar_wait_bounded(barP + 8 * s3(k), p3(k), kWaitLimit)) ok = false;
-                if (ok && !mbar_wait_bounded(barBC, par, kWaitLimit)) ok = false;
-                if (k >= 1 && ok && !mbar_wait_bounded(barC, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
+                if (k >= 1 && ok && !mbar_wait_bounded(barH, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
                 fence_after_sync();
                 const uint32_t colYs = kColYs0 + 64 * (uint32_t)sl;
                 const uint32_t aXWs = aXW + 16384 * (uint32_t)sl;
                 if constexpr (!STATE_ONLY) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tmem + kColCB, sdesc(aC + kk * 4096, 2048, 128), sdesc(aB + kk * 4096, 2048, 128), id_cb, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16(tmem + colYs, sdesc(aC + kk * 4096, 2048, 128), sdesc(aH + kk * 2048, 1024, 128), id_ys, kk > 0);
@@ -589,21 +666,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     mma_bf16(tmem + kColS, sdesc(aB + kk * 256, 128, 2048), sdesc(aXWs + kk * 2048, 1024, 128), id_s, kk > 0);
                 mma_commit(bar0);
                 mma_commit(barW + 8 * (uint32_t)sl);   // x'w of this block is free once they are done
-                // B'/C' are free once these MMAs are done: the next block's come in meanwhile
+                // B'/C' are free once all three products of this block are done (a commit covers
+                // every earlier MMA of this thread): the next block's come in meanwhile
                 if (k + 1 < nblk) {
                     if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
                     load_bc(k + 1);
                 }
-                if constexpr (!STATE_ONLY) {
-                    // M of this block is in TMEM once the consumer arrives on barC
-                    if (ok && !mbar_wait_bounded(barC, par, kWaitLimit)) ok = false;
-                    fence_after_sync();
-                    const uint32_t aXs = aX + 16384 * s3(k);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tmem + kColYi, tmem + kColM + kk * 8, sdesc(aXs + kk * 2048, 1024, 128), id_yi, kk > 0);
-                    mma_commit(bar1);
-                }
+            }
+            if constexpr (!STATE_ONLY) {
+                if (nblk > 0) mma_yi(nblk - 1);
             }
         }
     } else if constexpr (STATE_ONLY) {
@@ -611,7 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         float lam_tot = 0.0f;   // sum of delta*A over the row, log2 units
         for (int64_t k = 0; k < nblk; ++k) {
-            const int sl = (int)(k & 1);
             const uint32_t par = (uint32_t)(k & 1);
             if (ok && !mbar_wait_bounded(barP + 8 * s3(k), p3(k), kWaitLimit)) ok = false;
             if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
@@ -630,10 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             }
             fence_before_sync();
             named_sync(kBarCons, kThreads - kCons);
-            if (tid == kCons) {
-                mbar_arrive_local(barC);             // S^T read: the next block's MMA may overwrite it
-                mbar_arrive_local(barE2 + 8 * s3(k));   // the cumsum slot is free
-            }
+            if ((tid & 31) == 0) mbar_arrive_local(barH);   // S^T read: the next block's MMA may overwrite it
+            if (tid == kCons) mbar_arrive_local(barE2 + 8 * s3(k));   // the cumsum slot is free
         }
         float* fs = p.final_ssm + (sidx * p.H + h) * (int64_t)kP * kN;
 #pragma unroll
@@ -645,17 +713,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         const uint32_t aY = s_base + Lo::OFF_Y;
         // byte offset of 16-byte chunk c of token row r in the swizzled y tile
         auto ty_off = [](int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); };
-        // this thread's 32 channels of z for token crow of block kb: four 16-byte loads, issued
-        // well before the epilogue uses them (rows past the block's end read as zeros)
-        auto load_z = [&](int64_t kb, uint4* zr) {
+        // this thread's 32 channels of z for token crow of block kb: 16-byte loads nv of its four
+        // pieces from v0 on, issued well before the epilogue uses them (rows past the block's end
+        // read as zeros)
+        auto load_z = [&](int64_t kb, uint4* zr, int v0, int nv) {
             if (crow < blen(kb)) {
                 const uint4* zrow = reinterpret_cast<const uint4*>((const __nv_bfloat16*)p.z +
                                                                    (row0 + kb * kT + crow) * p.z_ld + h * kP + chalf * 32);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) zr[v] = zrow[v];
+                for (int v = 0; v < nv; ++v) zr[v0 + v] = zrow[v0 + v];
             } else {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) zr[v] = make_uint4(0u, 0u, 0u, 0u);
+                for (int v = 0; v < nv; ++v) zr[v0 + v] = make_uint4(0u, 0u, 0u, 0u);
             }
         };
         // this thread's 32 output channels of token crow into the y tile, then (thread kCons,
@@ -701,13 +770,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             tmem_wait_ld();
             store_y(kb, gv, scale, true);
         };
+        if (tid == kCons && nblk > 0) tma_prefetch_3d(&maps.z, h * kP, tmap_t0, tmap_b);
         for (int64_t k = 0; k < nblk; ++k) {
             const int64_t t0 = k * kT;
             const int len = blen(k);
             const int sl = (int)(k & 1);
             const uint32_t par = (uint32_t)(k & 1);
+            // z of the next block into L2 now, so that its loads below do not wait on HBM
+            if (tid == kCons && k + 1 < nblk) tma_prefetch_3d(&maps.z, h * kP, tmap_t0 + (int)((k + 1) * kT), tmap_b);
             if (ok && !mbar_wait_bounded(barP + 8 * s3(k), p3(k), kWaitLimit)) ok = false;
-            if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
+            if (ok && !mbar_wait_bounded(barCB, par, kWaitLimit)) ok = false;
             fence_after_sync();
             // expect the peers' sums of squares of block k (2 floats per row from every CTA)
             if constexpr (!SPLIT) {
@@ -717,12 +789,20 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             const float* dlb = s_dl + s3(k) * kT;
             const float* vb = s_v + s3(k) * kT;
             const float lam_end = lamb[kT - 1];
-            // masked, decayed M (row crow, columns chalf*64 .. +64) as bf16 pairs into TMEM
+            uint4 zr[4];
+            // masked, decayed M (row crow, columns chalf*64 .. +64) as bf16 pairs into TMEM. Every
+            // 8-column vector takes the same arithmetic (the causal mask is applied afterwards, to
+            // the vectors on or above the diagonal only), so the warps that hold the diagonal do
+            // not run several paths one after another.
             {
                 const int i = crow;
                 const float li = lamb[i];
+                // rows with lam_i > -96: exp2(lam_i - lam_j) = exp2(lam_i) * exp2(-lam_j), every
+                // factor a normal fp32 number; the choice uses only the row's own past, so outputs
+                // stay causal bit for bit
                 const bool fac = li > -96.0f;
-                const float ui = ex2(li);
+                const float2 u2 = splat2(ex2(li));
+                const float* gb = s_g + s3(k) * kT;
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     float cb[32];
@@ -732,39 +812,53 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         const int j0 = chalf * 64 + part * 32 + v * 8;
-                        if (j0 > i) {                 // above the diagonal: all zero
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) w[4 * v + e] = 0u;
-                        } else if (fac && j0 + 7 <= i) {   // wholly on or below it: no mask
+                        float2 m[4];
+                        if (fac) {
                             const float2* v2 = reinterpret_cast<const float2*>(vb + j0);
-                            const float2 u2 = splat2(ui);
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
-                                w[4 * v + e] = pack_f2(mul2(make_float2(cb[v * 8 + 2 * e], cb[v * 8 + 2 * e + 1]), mul2(u2, v2[e])));
-                        } else if (fac) {
-                            const float2* v2 = reinterpret_cast<const float2*>(vb + j0);
+                                m[e] = mul2(make_float2(cb[v * 8 + 2 * e], cb[v * 8 + 2 * e + 1]), mul2(u2, v2[e]));
+                        } else if (lamb[j0] - lamb[j0 + 7] < 100.0f) {
+                            // by 8-token segments: one exp2 per segment (it overflows only above the
+                            // diagonal, which the mask clears)
+                            const float2 sg = splat2(ex2(li - lamb[j0]));
+                            const float2* g2 = reinterpret_cast<const float2*>(gb + j0);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float2 m = mul2(make_float2(cb[v * 8 + 2 * e], cb[v * 8 + 2 * e + 1]), mul2(splat2(ui), v2[e]));
-                                if (j0 + 2 * e > i) m.x = 0.0f;
-                                if (j0 + 2 * e + 1 > i) m.y = 0.0f;
-                                w[4 * v + e] = pack_f2(m);
-                            }
+                            for (int e = 0; e < 4; ++e)
+                                m[e] = mul2(make_float2(cb[v * 8 + 2 * e], cb[v * 8 + 2 * e + 1]), mul2(sg, g2[e]));
                         } else {
+                            // a segment whose own decay leaves the fp32 range: element by element
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int j = j0 + 2 * e;
-                                const float mx = (j <= i) ? cb[v * 8 + 2 * e] * ex2(li - lamb[j]) * dlb[j] : 0.0f;
-                                const float my = (j + 1 <= i) ? cb[v * 8 + 2 * e + 1] * ex2(li - lamb[j + 1]) * dlb[j + 1] : 0.0f;
-                                w[4 * v + e] = pack_bf16x2(mx, my);
+                                m[e] = make_float2(cb[v * 8 + 2 * e] * ex2(li - lamb[j]) * dlb[j],
+                                                   cb[v * 8 + 2 * e + 1] * ex2(li - lamb[j + 1]) * dlb[j + 1]);
                             }
                         }
+                        if (j0 + 7 > i) {   // on or above the diagonal
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                if (j0 + 2 * e > i) m[e].x = 0.0f;
+                                if (j0 + 2 * e + 1 > i) m[e].y = 0.0f;
+                            }
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) w[4 * v + e] = pack_f2(m[e]);
                     }
                     tmem_st16(tmem + lane_base + kColM + chalf * 32 + part * 16, w);
                 }
             }
-            uint4 zr[4];
-            load_z(k, zr);   // in flight through the state update, the norm and the wait for M x'
+            // this warp's rows of M are in TMEM and its C'B'^T rows read: once all eight warps have
+            // arrived the control thread issues M x', which runs during the state update
+            tmem_wait_st();
+            fence_before_sync();
+            __syncwarp();
+            if ((tid & 31) == 0) mbar_arrive_local(barM);
+            load_z(k, zr, 0, 4);   // from L2 (prefetched a block ahead), in flight through the state update
+            // S^T of this block is in TMEM, and C'H^T of this block has read H^T
+            if (ok && !mbar_wait_bounded(bar0, par, kWaitLimit)) ok = false;
+            fence_after_sync();
+
             // state update H <- exp(lam_end) H + S and its bf16 copy for the next block
             {
                 float s_[32];
@@ -786,14 +880,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     *reinterpret_cast<uint4*>(sH + canon_off(crow, chalf * 32 + 8 * v, kP)) = u;
                 }
             }
-            tmem_wait_st();
+            // S^T read and H^T of block k+1 written (generic stores made visible to the tensor
+            // cores): the next block's MMAs may start
             fence_async_smem();
             fence_before_sync();
-            if (tid == kCons) bulk_wait_read_all();   // the previous y store has left the y tile
-            named_sync(kBarCons, kThreads - kCons);
-            // M written, C'B'^T and S^T read, H^T of block k+1 written: the control thread issues
-            // M x' of this block, then the next block's MMAs
-            if (tid == kCons) mbar_arrive_local(barC);
+            __syncwarp();
+            if ((tid & 31) == 0) mbar_arrive_local(barH);
             if constexpr (!SPLIT) {
                 if (k >= 1) finish_norm(k - 1);   // overlaps the MMA M x' of this block
             }
@@ -843,6 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 }
             }
             fence_before_sync();
+            if (tid == kCons) bulk_wait_read_all();   // the last y store has left the y tile
             named_sync(kBarCons, kThreads - kCons);
             if (tid == kCons) mbar_arrive_local(barE2 + 8 * s3(k));   // the x' and cumsum slots are free
             if constexpr (SPLIT) store_y(k, gt, 1.0f, false);
@@ -952,30 +1045,15 @@ EncodeTiledFn encode_tiled_fn()
     return fn;
 }
 
-// [b][L][width] bf16 rows of `ld` elements viewed as [b][width/8 vectors][L][8]; boxes of
-// 8 channels x `rows` tokens x `nvec` vectors x 1 sequence land as [vector][token][8].
-bool encode_rows(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b, int nvec, int rows)
-{
-    EncodeTiledFn enc = encode_tiled_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[4] = {8, (cuuint64_t)L, (cuuint64_t)(width / 8), (cuuint64_t)b};
-    const cuuint64_t strides[3] = {(cuuint64_t)(ld * 2), 16, (cuuint64_t)(L * ld * 2)};
-    const cuuint32_t box[4] = {8, (cuuint32_t)rows, (cuuint32_t)nvec, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// [b][L][width] bf16 rows of `ld` elements; boxes of 64 channels x 128 tokens x 1 sequence,
+// [b][L][width] bf16 rows of `ld` elements; boxes of 64 channels x `rows` tokens x 1 sequence,
 // 128-byte swizzled in shared memory.
-bool encode_tile(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b)
+bool encode_tile(CUtensorMap* m, const void* base, int64_t width, int64_t ld, int64_t L, int64_t b, int rows)
 {
     EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)L, (cuuint64_t)b};
     const cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(L * ld * 2)};
-    const cuuint32_t box[3] = {(cuuint32_t)kP, (cuuint32_t)kT, 1};
+    const cuuint32_t box[3] = {(cuuint32_t)kP, (cuuint32_t)rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -1004,10 +1082,10 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     // packed sequences: one row of all the packed tokens
     const int64_t mL = p.L, mb = p.cu_seqlens ? 1 : p.b;
     if (p.L > 0) {   // no block, no load: the maps stay unused
-        if (!encode_rows(&maps.x, p.x, p.HP(), p.x_ld, mL, mb, kVX, kStageRows) ||
-            !encode_rows(&maps.bc, p.bcp, 2 * p.GN(), 2 * p.GN(), mL, mb, kN / 8, kT))
+        if (!encode_tile(&maps.x, p.x, p.HP(), p.x_ld, mL, mb, kStageRows)) return cudaErrorInvalidValue;
+        if (!STATE_ONLY && (!encode_tile(&maps.y, p.y, p.HP(), p.y_ld, mL, mb, kT) ||
+                            !encode_tile(&maps.z, p.z, p.HP(), p.z_ld, mL, mb, kT)))
             return cudaErrorInvalidValue;
-        if (!STATE_ONLY && !encode_tile(&maps.y, p.y, p.HP(), p.y_ld, mL, mb)) return cudaErrorInvalidValue;
     }
     e = cudaFuncSetAttribute(ssd_prefill_ws_kernel<R, SPLIT, STATE_ONLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Lo::TOTAL);
