@@ -178,108 +178,97 @@ __device__ __forceinline__ float scan128(float v, float* tot)
     return v + off;
 }
 
-// The sequence that packed token row t belongs to: its index, first row, length, state slot,
-// and whether it starts from the initial conv state given.
-struct SeqOf {
-    int64_t s, start, len, slot;
-    bool init;
-};
-__device__ __forceinline__ SeqOf seq_of(const PrefillParams& p, int64_t t)
+// SiLU(conv) of the B and C channels (the first nch of the 2*G*N), once per token for all the
+// heads that read them, into the workspace as one 32 KB chunk per (128-token block of a
+// sequence, matrix, group) in the MMA operand layout (prefill_bc_blocks), so the main kernel
+// fetches each with one contiguous copy. One CTA per (block slot, 64 channels): the block's raw
+// rows and its 3-row halo (the sequence's initial conv state before its first token, zeros
+// without one) are loaded with coalesced 16-byte loads into a padded tile, and each 8-channel
+// vector's [128 tokens][8] slab is written as one contiguous 2 KB run, zeros past the end of
+// the sequence.
+constexpr int kBcRows = kT + 3, kBcPitch = 9;   // tile rows (block + halo), 16-byte pieces per row
+__global__ void __launch_bounds__(256) bc_conv_kernel(PrefillParams p, int nch)
 {
-    SeqOf r;
-    if (!p.cu_seqlens) {
-        r.s = t / p.L;
-        r.start = r.s * p.L;
-        r.len = p.L;
-        r.slot = r.s;
-        r.init = p.init_conv != nullptr;
-        return r;
-    }
-    int64_t lo = 0, hi = p.b - 1;   // the last sequence i with cu_seqlens[i] <= t
+    __shared__ uint4 tile[kBcRows * kBcPitch];
+    __shared__ float4 wsm[64];
+    __shared__ float bsm[64];
+    const int64_t GN = p.GN(), HP = p.HP(), Cc = p.Cc();
+    const int64_t slot_blk = blockIdx.x;
+    const int64_t c0 = (int64_t)blockIdx.y * 64;   // first channel within [B | C]
+    const int tid = threadIdx.x;
+    // the sequence whose blocks hold this slot: the last s with s + start_s / 128 <= slot_blk
+    auto start_of = [&](int64_t s) { return p.cu_seqlens ? (int64_t)p.cu_seqlens[s] : s * p.L; };
+    int64_t lo = 0, hi = p.b - 1;
     while (lo < hi) {
         const int64_t mid = (lo + hi + 1) / 2;
-        if ((int64_t)p.cu_seqlens[mid] <= t) lo = mid;
+        if (mid + start_of(mid) / kT <= slot_blk) lo = mid;
         else hi = mid - 1;
     }
-    r.s = lo;
-    r.start = p.cu_seqlens[lo];
-    r.len = (int64_t)p.cu_seqlens[lo + 1] - r.start;
-    r.slot = p.slot_idx ? (int64_t)p.slot_idx[lo] : lo;
-    r.init = p.init_conv != nullptr && (!p.has_init || p.has_init[lo] != 0);
-    return r;
-}
-
-// SiLU(conv) of the B and C channels (the first nch of the 2*G*N), once per token for all the
-// heads that read them. One thread per (8-channel vector, run of kBcRun tokens): its taps in
-// registers and the run's kBcRun + 3 raw rows loaded at once; before a sequence's first token
-// the window reads its initial conv state (zeros without one). Output in the workspace as one
-// 32 KB chunk per (128-token block of a sequence, matrix, group) in the MMA operand layout
-// (prefill_bc_blocks), so the main kernel fetches each with one contiguous copy.
-constexpr int kBcRun = 4;
-__global__ void __launch_bounds__(256, 2) bc_conv_kernel(PrefillParams p, int nch)
-{
-    const int64_t GN = p.GN(), HP = p.HP(), Cc = p.Cc(), rows = p.rows();
-    const int64_t v = (int64_t)blockIdx.x * 8 + (threadIdx.x & 7);
-    const int64_t t0 = ((int64_t)blockIdx.y * 32 + (threadIdx.x >> 3)) * kBcRun;
-    if (v * 8 >= nch || t0 >= rows) return;
-    const int64_t c0 = v * 8;                       // channel within [B | C]
+    const int64_t s = lo, start = start_of(s);
+    const int64_t len = p.cu_seqlens ? (int64_t)p.cu_seqlens[s + 1] - start : p.L;
+    const int64_t k = slot_blk - (s + start / kT);
+    if (k < 0 || k * kT >= len) return;   // a slot no block of any sequence uses
+    const int64_t slot = p.cu_seqlens && p.slot_idx ? (int64_t)p.slot_idx[s] : s;
+    const bool init = p.init_conv != nullptr && (!p.cu_seqlens || !p.has_init || p.has_init[s] != 0);
     const bool isC = c0 >= GN;
-    const int64_t cg = (isC ? c0 - GN : c0) / kN, cv = ((isC ? c0 - GN : c0) % kN) / 8;   // group, vector
     const __nv_bfloat16* src = (const __nv_bfloat16*)(isC ? p.C : p.B) + (isC ? c0 - GN : c0);
     const int64_t ld = isC ? p.C_ld : p.B_ld;
-    float w[8][4], bb[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float4 wv = *reinterpret_cast<const float4*>(p.conv_w + (HP + c0 + e) * 4);
-        w[e][0] = wv.x; w[e][1] = wv.y; w[e][2] = wv.z; w[e][3] = wv.w;
-        bb[e] = p.conv_b[HP + c0 + e];
+    if (tid < 64) {
+        wsm[tid] = *reinterpret_cast<const float4*>(p.conv_w + (HP + c0 + tid) * 4);
+        bsm[tid] = p.conv_b[HP + c0 + tid];
     }
-    // every raw row the run's windows can touch, loaded up front (rows outside the call as
-    // zeros); whether a row is a raw input or the sequence's initial state is decided per token
-    uint4 raw[kBcRun + 3];
+    // tile row r holds token k*128 + r - 3 of the sequence; every load of a thread is issued
+    // before the first one is stored
+    constexpr int kLoads = (kBcRows * 8 + 255) / 256;
+    uint4 val[kLoads];
 #pragma unroll
-    for (int j = 0; j < kBcRun + 3; ++j) {
-        const int64_t r = t0 - 3 + j;
-        raw[j] = (r >= 0 && r < rows) ? *reinterpret_cast<const uint4*>(src + r * ld) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < kLoads; ++i) {
+        const int e = tid + 256 * i;
+        const int r = e / 8, v = e % 8;
+        const int64_t tok = k * kT + r - 3;
+        val[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (e < kBcRows * 8 && tok >= 0 && tok < len) val[i] = *reinterpret_cast<const uint4*>(src + (start + tok) * ld + v * 8);
     }
-    SeqOf sq = seq_of(p, t0);
 #pragma unroll
-    for (int u = 0; u < kBcRun; ++u) {
-        const int64_t t = t0 + u;
-        if (t >= rows) break;
-        if (t >= sq.start + sq.len) sq = seq_of(p, t);   // the run crossed into the next sequence
-        float acc[8];
+    for (int i = 0; i < kLoads; ++i) {
+        const int e = tid + 256 * i;
+        const int r = e / 8, v = e % 8;
+        const int64_t tok = k * kT + r - 3;
+        if (e < kBcRows * 8 && tok < 0 && init) {   // the initial conv state, oldest first
+            __nv_bfloat16 hv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = bb[e];
+            for (int q = 0; q < 8; ++q)
+                hv[q] = ((const __nv_bfloat16*)p.init_conv)[(slot * Cc + HP + c0 + v * 8 + q) * 3 + (tok + 3)];
+            val[i] = *reinterpret_cast<const uint4*>(hv);
+        }
+        if (e < kBcRows * 8) tile[r * kBcPitch + v] = val[i];
+    }
+    __syncthreads();
+    const int64_t mat = isC ? 1 : 0, cw = isC ? c0 - GN : c0;   // channel within its matrix
+    __nv_bfloat16* chunk = (__nv_bfloat16*)p.bcp + ((slot_blk * 2 + mat) * p.G + cw / kN) * (int64_t)(kT * kN);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {   // tap j multiplies token t - 3 + j
-            const int64_t r = t - 3 + j;
-            float in[8];
-            if (r >= sq.start) {
-                unpack_bf16x8(raw[u + j], in);
-            } else {
-                const int64_t k = r - sq.start + 3;   // 0..2: the initial conv state, oldest first
+    for (int i = 0; i < 4; ++i) {
+        const int o = tid + 256 * i;
+        const int v = o / kT, t = o % kT;   // consecutive threads: consecutive tokens of one vector
+        float out[8];
+        if (k * kT + t < len) {
+            float acc[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    in[e] = sq.init ? __bfloat162float(((const __nv_bfloat16*)p.init_conv)[(sq.slot * Cc + HP + c0 + e) * 3 + k])
-                                    : 0.0f;
+            for (int q = 0; q < 8; ++q) acc[q] = bsm[v * 8 + q];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {   // tap j multiplies token t - 3 + j (tile row t + j)
+                float in[8];
+                unpack_bf16x8(tile[(t + j) * kBcPitch + v], in);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = fmaf((&wsm[v * 8 + q].x)[j], in[q], acc[q]);
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[e][j], in[e], acc[e]);
-        }
-        float o[8];
+            for (int q = 0; q < 8; ++q) out[q] = tc::silu_fast(acc[q]);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = tc::silu_fast(acc[e]);
-        // block k of sequence s, row pos of this vector's [128 tokens][8] slab of the chunk
-        const int64_t pos = t - sq.start;
-        __nv_bfloat16* slab = (__nv_bfloat16*)p.bcp +
-                              ((((sq.s + sq.start / kT + pos / kT) * 2 + (isC ? 1 : 0)) * p.G + cg) * (kN / 8) + cv) * (kT * 8);
-        store_vec<__nv_bfloat16>(slab + (pos % kT) * 8, o);
-        // the rows of a sequence's last block past its end are zeros (the MMAs read the whole block)
-        if (pos == sq.len - 1) {
-            for (int64_t r = pos % kT + 1; r < kT; ++r)
-                *reinterpret_cast<uint4*>(slab + r * 8) = make_uint4(0u, 0u, 0u, 0u);
+            for (int q = 0; q < 8; ++q) out[q] = 0.0f;
         }
+        store_vec<__nv_bfloat16>(chunk + (((cw % kN) / 8 + v) * kT + t) * 8, out);
     }
 }
 
@@ -1066,7 +1055,7 @@ cudaError_t launch_bc_conv(const PrefillParams& p, int nch, cudaStream_t st)
     const int64_t rows = p.rows();
     if (rows == 0) return cudaSuccess;
     LaunchScope ls("tc_bc_conv", st);
-    const dim3 grid((unsigned)((nch / 8 + 7) / 8), (unsigned)((rows + 32 * kBcRun - 1) / (32 * kBcRun)));
+    const dim3 grid((unsigned)prefill_bc_blocks(p.b, rows), (unsigned)(nch / 64));
     bc_conv_kernel<<<grid, 256, 0, st>>>(p, nch);
     return cudaGetLastError();
 }
