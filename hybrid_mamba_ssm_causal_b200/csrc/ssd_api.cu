@@ -498,7 +498,9 @@ const char* ssd_status_string(ssd_status s)
     case SSD_ERR_CUDA: return "CUDA launch or runtime error";
     case SSD_ERR_TIMEOUT: return "a bounded device-side wait timed out";
     case SSD_ERR_TOO_LARGE: return "problem needs more scratch than the fixed static workspace holds";
-    case SSD_ERR_DEVICE: return "a kernel could not start its work (its shared memory base was misaligned)";
+    case SSD_ERR_DEVICE:
+        return "a kernel could not start its work (its shared memory base was misaligned), or, in the "
+               "bounds-checked build, an index fell outside its buffer";
     }
     return "unknown status";
 }

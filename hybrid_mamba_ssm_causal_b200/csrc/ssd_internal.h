@@ -20,9 +20,24 @@ enum DeviceStatus : int {
     kDevOk = 0,
     kDevTimeout = 1,          // a bounded wait (mbarrier, peer copy, tensor-core commit) gave up
     kDevSmemMisaligned = 2,   // the dynamic shared memory base lacked the alignment the kernel needs
+    kDevBounds = 3,           // (bounds-checked build) an index fell outside its buffer; access skipped
 };
 #ifdef __CUDACC__
 __device__ __forceinline__ void set_device_status(int* status, int code) { atomicCAS(status, 0, code); }
+// SSD_IN_BOUNDS(status, cond): in the bounds-checked build (compiled with -DSSD_DEBUG_BOUNDS,
+// libssd_mixer_debug.so) a false cond records kDevBounds in the status word and the guarded
+// access is skipped, so a bad index is reported instead of faulting; in the normal build it is
+// `true` and cond is not evaluated.
+#ifdef SSD_DEBUG_BOUNDS
+__device__ __forceinline__ bool ssd_in_bounds(int* status, bool ok)
+{
+    if (!ok) set_device_status(status, kDevBounds);
+    return ok;
+}
+#define SSD_IN_BOUNDS(status, cond) ::ssd::ssd_in_bounds((status), (cond))
+#else
+#define SSD_IN_BOUNDS(status, cond) true
+#endif
 #endif
 // Clears the status word of a call's workspace on its stream.
 inline cudaError_t clear_device_status(int* status, cudaStream_t st)
@@ -165,7 +180,7 @@ cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream);
 // layout [16 vectors of 8 channels][128 tokens][8]. Sequences never share a chunk, and
 // prefill_bc_blocks(b, rows) = b + rows / 128 + 1 bounds the block index.
 constexpr int64_t kBcBlockTokens = 128;
-inline size_t prefill_bc_blocks(int64_t b, int64_t rows) { return (size_t)(b + rows / kBcBlockTokens + 1); }
+SSD_HD inline size_t prefill_bc_blocks(int64_t b, int64_t rows) { return (size_t)(b + rows / kBcBlockTokens + 1); }
 int prefill_ws_partials_per_head();
 
 // H_in(r) of a sequence split into pieces: init (NULL = zeros) carried through pieces 0..r-1.

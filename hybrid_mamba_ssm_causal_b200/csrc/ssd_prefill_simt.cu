@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(PrefillParams p)
         __syncthreads();
     }
     float* S = p.states + (((bi * p.nc + c) * p.H + h) * (int64_t)P) * N;
+    if (!SSD_IN_BOUNDS(p.status, bi < p.b && c < p.nc && h < p.H)) return;
 #pragma unroll
     for (int i = 0; i < RP; ++i)
 #pragma unroll
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(256) chunk_scan_kernel(PrefillParams p)
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         const int i = i0 + ty + 16 * a;
-        if (i >= len) continue;
+        if (i >= len || !SSD_IN_BOUNDS(p.status, t0 + i < p.L)) continue;
         const float el = expf(s.lam[i]);
         float* yo = p.ypre + (bi * p.L + t0 + i) * HP + (int64_t)h * P;
 #pragma unroll

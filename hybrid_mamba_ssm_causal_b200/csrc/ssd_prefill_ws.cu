@@ -227,7 +227,8 @@ __global__ void __launch_bounds__(256) bc_conv_kernel(PrefillParams p, int nch)
         const int r = e / 8, v = e % 8;
         const int64_t tok = k * kT + r - 3;
         val[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (e < kBcRows * 8 && tok >= 0 && tok < len) val[i] = *reinterpret_cast<const uint4*>(src + (start + tok) * ld + v * 8);
+        if (e < kBcRows * 8 && tok >= 0 && tok < len && SSD_IN_BOUNDS(p.status, start + tok < p.rows()))
+            val[i] = *reinterpret_cast<const uint4*>(src + (start + tok) * ld + v * 8);
     }
 #pragma unroll
     for (int i = 0; i < kLoads; ++i) {
@@ -268,7 +269,8 @@ __global__ void __launch_bounds__(256) bc_conv_kernel(PrefillParams p, int nch)
 #pragma unroll
             for (int q = 0; q < 8; ++q) out[q] = 0.0f;
         }
-        store_vec<__nv_bfloat16>(chunk + (((cw % kN) / 8 + v) * kT + t) * 8, out);
+        if (SSD_IN_BOUNDS(p.status, (slot_blk * 2 + mat) * p.G + cw / kN < (int64_t)prefill_bc_blocks(p.b, p.rows()) * 2 * p.G))
+            store_vec<__nv_bfloat16>(chunk + (((cw % kN) / 8 + v) * kT + t) * 8, out);
     }
 }
 
@@ -416,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 dl = softplus(__uint_as_float(dt_next << 16) + bias);
                 a2 = dl * A2;
             }
-            if (kb + 1 < nblk && (kb + 1) * kT + tok < seqlen)
+            if (kb + 1 < nblk && (kb + 1) * kT + tok < seqlen &&
+                SSD_IN_BOUNDS(p.status, row0 + (kb + 1) * kT + tok < p.rows()))
                 dt_next = gdt16[(row0 + (kb + 1) * kT + tok) * p.dt_ld + h];
             const float lam = scan128(a2, s_scan);
             s_lam[slb * kT + tok] = lam;
@@ -511,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 for (int64_t kb = 0; kb < XBUF && kb < nblk; ++kb) load_x(kb);
             }
             if (tid >= kScan0) {
-                if (tok < seqlen) dt_next = gdt16[(row0 + tok) * p.dt_ld + h];
+                if (tok < seqlen && SSD_IN_BOUNDS(p.status, row0 + tok < p.rows())) dt_next = gdt16[(row0 + tok) * p.dt_ld + h];
                 scan_block(0);
             }
         }
@@ -607,10 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             auto load_bc = [&](int64_t kb) {
                 constexpr uint32_t kChunk = (uint32_t)kT * kN * 2;
                 mbar_arrive_expect_tx(barBC, (STATE_ONLY ? 1u : 2u) * kChunk);
-                const unsigned char* cB =
-                    (const unsigned char*)p.bcp + (((bi + row0 / kT + kb) * 2) * p.G + g) * (int64_t)kChunk;
-                bulk_load(aB, cB, kChunk, barBC);
-                if (!STATE_ONLY) bulk_load(aC, cB + (int64_t)p.G * kChunk, kChunk, barBC);
+                const int64_t ci = ((bi + row0 / kT + kb) * 2) * p.G + g;
+                const unsigned char* cB = (const unsigned char*)p.bcp + ci * (int64_t)kChunk;
+                if (SSD_IN_BOUNDS(p.status, ci + p.G < (int64_t)prefill_bc_blocks(p.b, p.rows()) * 2 * p.G)) {
+                    bulk_load(aB, cB, kChunk, barBC);
+                    if (!STATE_ONLY) bulk_load(aC, cB + (int64_t)p.G * kChunk, kChunk, barBC);
+                } else {   // nothing lands: complete the expected bytes so no wait is left hanging
+                    mbar_arrive_expect_tx(barBC, 0u);
+                }
             };
             if (nblk > 0) load_bc(0);
             // M x' of block kb, once every consumer warp has written its rows of M
@@ -706,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         // pieces from v0 on, issued well before the epilogue uses them (rows past the block's end
         // read as zeros)
         auto load_z = [&](int64_t kb, uint4* zr, int v0, int nv) {
-            if (crow < blen(kb)) {
+            if (crow < blen(kb) && SSD_IN_BOUNDS(p.status, row0 + kb * kT + crow < p.rows())) {
                 const uint4* zrow = reinterpret_cast<const uint4*>((const __nv_bfloat16*)p.z +
                                                                    (row0 + kb * kT + crow) * p.z_ld + h * kP + chalf * 32);
 #pragma unroll
@@ -736,7 +743,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                     w[e] = pack_f2(norm ? mul2(mul2(gg, splat2(scale)), nw2[4 * v + e]) : gg);
                 }
                 if (!rows_only) *reinterpret_cast<uint4*>(ty + ty_off(crow, chalf * 4 + v)) = make_uint4(w[0], w[1], w[2], w[3]);
-                else if (crow < blen(kb)) yrow[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                else if (crow < blen(kb) && SSD_IN_BOUNDS(p.status, row0 + kb * kT + crow < p.rows()))
+                    yrow[v] = make_uint4(w[0], w[1], w[2], w[3]);
             }
             if (rows_only) return;
             fence_async_smem();
@@ -912,7 +920,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 }
                 const float ss = ss2.x + ss2.y;
                 if constexpr (SPLIT) {
-                    if (i < len) p.ssp[((row0 + t0 + i) * p.H + h) * 2 + chalf] = ss;
+                    if (i < len && SSD_IN_BOUNDS(p.status, row0 + t0 + i < p.rows()))
+                        p.ssp[((row0 + t0 + i) * p.H + h) * 2 + chalf] = ss;
                 } else {
                     const uint32_t nsl = (uint32_t)(k % 3);
                     const uint32_t dst = smem_u32(s_red + ((nsl * R + q) * 2 + chalf) * 128 + i);

@@ -26,7 +26,9 @@ from dataclasses import dataclass
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libssd_mixer.so")
+# the library the binding opens: libssd_mixer.so, or another build of it (the bounds-checked
+# libssd_mixer_debug.so) named by SSD_MIXER_LIBRARY
+LIB_PATH = os.environ.get("SSD_MIXER_LIBRARY") or os.path.join(HERE, "libssd_mixer.so")
 
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT, SSD_ERR_TOO_LARGE, SSD_ERR_DEVICE = range(7)
 SSD_MIXER_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024

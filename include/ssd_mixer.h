@@ -73,7 +73,8 @@ typedef enum ssd_status {
     SSD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
     SSD_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (status word) */
     SSD_ERR_TOO_LARGE = 5,    /* needs more scratch than the fixed static workspace */
-    SSD_ERR_DEVICE = 6,       /* a kernel could not start its work (status word) */
+    SSD_ERR_DEVICE = 6,       /* a kernel could not start its work, or (bounds-checked build)
+                                 an index fell outside its buffer (status word) */
 } ssd_status;
 
 typedef enum ssd_dtype {
@@ -412,8 +413,9 @@ SSD_API ssd_status ssd_mixer_backward(const ssd_dims* dims,
  * `workspace` (the last call that used it clears it on its stream before its first kernel,
  * and its kernels record the first failure). Synchronises `stream`. Returns SSD_OK;
  * SSD_ERR_TIMEOUT if a bounded device-side wait gave up; SSD_ERR_DEVICE if a kernel found
- * its dynamic shared memory base misaligned and did no work. In both error cases that
- * call's outputs are invalid. */
+ * its dynamic shared memory base misaligned and did no work, or, in the bounds-checked build
+ * (libssd_mixer_debug.so), an index fell outside its buffer and its access was skipped. In
+ * every error case that call's outputs are invalid. */
 SSD_API ssd_status ssd_mixer_workspace_status(const void* workspace, void* stream);
 
 /* Self-test of the failure path that every bounded device-side wait in the library takes
