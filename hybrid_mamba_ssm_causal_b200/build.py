@@ -39,7 +39,8 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale(lib: str = LIB) -> bool:
+def _stale(lib: str | None = None) -> bool:
+    lib = lib or LIB
     if not os.path.exists(lib):
         return True
     t = os.path.getmtime(lib)
