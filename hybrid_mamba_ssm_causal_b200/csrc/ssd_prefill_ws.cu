@@ -7,7 +7,8 @@
 //   lam_i = inclusive sum of delta*A (log2 units), CB = C' B'^T, Ys = C' H^T,
 //   S^T = B'^T (x' w) with w_j = exp(lam_end - lam_j) delta_j,
 //   M_ij = CB_ij exp(lam_i - lam_j) delta_j (j <= i), Yi = M x',
-//   y = Yi + exp(lam_i) Ys + D x',  g = y SiLU(z),  out = g / rms_group(g) * norm_w,
+//   y = Yi + exp(lam_i) Ys + D x',  g = y SiLU(z),  out = g / rms_group(g) * norm_w
+//   (for groups held by a cluster D sits on M's diagonal, so Yi already holds D x'),
 //   H <- exp(lam_end) H + S.
 //
 // Two kernels per call (three when the norm group is wider than a cluster):
@@ -837,7 +838,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                             for (int e = 0; e < 4; ++e) {
                                 if (j0 + 2 * e > i) m[e].x = 0.0f;
                                 if (j0 + 2 * e + 1 > i) m[e].y = 0.0f;
+                                // groups held by a cluster: the D skip rides on the diagonal, so M x'
+                                // gives D x'_i too and the epilogue reads no x' (the wide-group variant
+                                // is at its register limit and keeps D x' in the epilogue)
+                                if constexpr (!SPLIT) {
+                                    if (j0 + 2 * e == i) m[e].x += Dh;
+                                    if (j0 + 2 * e + 1 == i) m[e].y += Dh;
+                                }
                             }
+                        } else if (!SPLIT && j0 + 7 == i) {
+                            m[3].y += Dh;
                         }
 #pragma unroll
                         for (int e = 0; e < 4; ++e) w[4 * v + e] = pack_f2(m[e]);
@@ -892,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             float gt[32];
             {
                 const int i = crow;
-                const float2 el = splat2(ex2(lamb[i])), d2 = splat2(Dh);
+                const float2 el = splat2(ex2(lamb[i])), d2 = splat2(SPLIT ? Dh : 0.0f);
                 const unsigned char* sX = smem + Lo::OFF_X + s3(k) * 16384;
                 float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
@@ -904,13 +914,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
 #pragma unroll
                     for (int vv = 0; vv < 2; ++vv) {
                         const int v = hf * 2 + vv;
-                        const uint4 xw = *reinterpret_cast<const uint4*>(sX + canon_off(i, chalf * 32 + 8 * v, kP));
+                        const uint4 xw = SPLIT ? *reinterpret_cast<const uint4*>(sX + canon_off(i, chalf * 32 + 8 * v, kP))
+                                               : make_uint4(0u, 0u, 0u, 0u);
                         const uint4 zv = zr[v];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int c = 8 * vv + 2 * e;
                             float2 y = fma2(el, make_float2(ys[c], ys[c + 1]), make_float2(yi[c], yi[c + 1]));
-                            y = fma2(d2, bf2_to_f2((&xw.x)[e]), y);
+                            if constexpr (SPLIT) y = fma2(d2, bf2_to_f2((&xw.x)[e]), y);
                             const float2 gg = mul2(y, silu2(bf2_to_f2((&zv.x)[e])));
                             gt[8 * v + 2 * e] = gg.x;
                             gt[8 * v + 2 * e + 1] = gg.y;
