@@ -642,10 +642,32 @@ def main():
             return rank_max(f0.elapsed_time(f1) / steps)
 
         ems = e2e_timed(e2e_step, a.steps, max(3, min(a.warmup, 5)))
+
+        def h2d_step(_i):   # the step's host-to-device copies alone, on the same copy stream
+            with torch.cuda.stream(s_in):
+                for k in (0, 1):
+                    for n in seq_keys:
+                        half(X[n], k).copy_(half(host[n], k), non_blocking=True)
+                for n in seq_keys:
+                    DQ[n].copy_(hdec[n], non_blocking=True)
+
+        def copies_timed(fn, steps):
+            fn(0)
+            torch.cuda.synchronize()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(s_in)
+            for i in range(steps):
+                fn(i)
+            f1.record(s_in)
+            torch.cuda.synchronize()
+            return rank_max(f0.elapsed_time(f1) / steps)
+
+        h2d_ms = copies_timed(h2d_step, max(3, min(a.steps, 10)))
         e2e = {"value": job_value(world, tok_step, ems), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": ems,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "h2d_only_ms_per_step": h2d_ms,
                "how": "pinned host buffers; each call's inputs copied in on a copy stream, y copied out on "
-                      "another, overlapped with the other call's compute"}
+                      "another, overlapped with the other call's compute; h2d_only_ms_per_step times the "
+                      "host-to-device copies of a step alone"}
         del host, hy
     del X, y
 
