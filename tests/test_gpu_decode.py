@@ -88,3 +88,19 @@ def test_decode_small_shapes_with_permuted_slots(act, H, P, G, N):
     assert_close("y", ys.permute(1, 0, 2), ref["y"], tol)
     assert_close("ssm_state", ssm, ref["final_ssm"], tol)
     assert_close("conv_state", conv, ref["final_conv"], tol)
+
+
+@pytest.mark.parametrize("b,H,G", [(1, 256, 8), (3, 16, 2), (4, 4, 2)])
+def test_decode_small_batches_split_groups_over_clusters(b, H, G):
+    """Few sequences: each group's heads are split over a cluster of CTAs (8, 8 and 2 CTAs per
+    group here) that exchange their partial sums of squares through distributed shared memory.
+    The first case is the decode token of the long_bf16 step."""
+    w = WORKLOADS["decode_bf16"].with_(batch=b, nheads=H, ngroups=G)
+    inp = make_decode_inputs(w, steps=12, seed=9)
+    slots = list(reversed(range(b))) if b > 1 else None
+    ys, ssm, conv = run_steps(w, inp, 12, b, slot_idx=slots, nslots=b)
+    ref = oracle_as_prefill(w, inp, 12, b)
+    tol = TOL[w.act]
+    assert_close("y", ys.permute(1, 0, 2), ref["y"], tol)
+    assert_close("ssm_state", ssm, ref["final_ssm"], tol)
+    assert_close("conv_state", conv, ref["final_conv"], tol)
