@@ -48,7 +48,7 @@ METRIC = "Mamba-2 SSD mixer prefill tokens/s & decode steps/s; % of HBM roofline
 HEADLINE = "long_bf16"
 SUB_PREFILL = ("tiny_f32", "small_bf16", "mid_bf16")
 L2_BYTES = 126 * 2**20
-TRAFFIC_FILE = "profiles/dram_traffic_per_launch.json"
+TRAFFIC_FILE = "profiles/dram_traffic_per_call.json"
 # model width of the layer sub-record: Nemotron-3 Nano, whose Mamba mixer has the mid workload's
 # 64 heads x 64 (Modalities PR #459, commit notes: dimension 2688)
 LAYER_D_MODEL = 2688
@@ -232,9 +232,10 @@ def sources_sha256(name: str) -> str:
 
 
 def measured_traffic(name: str, workload: str, path: str | None = None):
-    """dram__bytes_read.sum + dram__bytes_write.sum per launch of kernel ``name`` on
-    ``workload``, from the committed ncu figures (a small JSON file beside the summaries), or
-    None when there is no entry or the kernel's sources changed since the capture."""
+    """dram__bytes_read.sum + dram__bytes_write.sum per call of kernel ``name`` on ``workload``
+    (summed over the call's launches), from the committed ncu figures (a small JSON file beside
+    the summaries), or None when there is no entry or the kernel's sources changed since the
+    capture."""
     try:
         with open(path or os.path.join(ROOT, TRAFFIC_FILE)) as f:
             data = json.load(f)
@@ -245,7 +246,7 @@ def measured_traffic(name: str, workload: str, path: str | None = None):
             if name not in KERNEL_SOURCES or e.get("kernel_sources_sha256") != sources_sha256(name):
                 return None
             try:
-                return float(e["traffic_bytes_per_launch"])
+                return float(e["traffic_bytes_per_call"])
             except (KeyError, TypeError, ValueError):
                 return None
     return None
@@ -440,18 +441,22 @@ def profiled(lib, fn, n):
     return out
 
 
-def roofline_of(per_kernel: dict, bytes_of, hbm: float, peak_src: str, traffic=None):
-    """Roofline of the kernel with the largest device time: algorithmic bytes per launch over
-    its average launch time, against the measured copy bandwidth."""
+def roofline_of(per_kernel: dict, bytes_of, hbm: float, peak_src: str, traffic=None, calls=None):
+    """Roofline of the kernel with the largest device time: algorithmic bytes per call over its
+    device time per call (the sum of the call's launches: the main prefill kernel runs a call
+    as several launches when its rows are split into pieces), against the measured copy
+    bandwidth. ``calls``: the calls in the profiled region (default: one per launch)."""
     if not per_kernel:
         return None
     name, (tot_ms, n) = max(per_kernel.items(), key=lambda kv: kv[1][0])
     kb = bytes_of(name)
-    avg_ms = tot_ms / n
-    ach = kb / (avg_ms * 1e-3) / 1e9 if kb else None
+    nc = calls or n
+    call_ms = tot_ms / nc
+    ach = kb / (call_ms * 1e-3) / 1e9 if kb else None
     return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
             "frac": (ach / hbm) if ach else None, "traffic": traffic(name) if traffic else None,
-            "peak_source": peak_src, "avg_launch_us": avg_ms * 1e3, "algorithmic_bytes_per_launch": kb,
+            "peak_source": peak_src, "us_per_call": call_ms * 1e3, "launches_per_call": n / nc,
+            "avg_launch_us": tot_ms / n * 1e3, "algorithmic_bytes_per_call": kb,
             "share_of_kernel_time": tot_ms / sum(v[0] for v in per_kernel.values())}
 
 
@@ -566,9 +571,10 @@ def main():
             return call_bytes
         return kernel_bytes(name, w, w.batch, L1)
 
-    roofline = roofline_of(per_kernel, head_bytes, hbm, peak_src, lambda n: measured_traffic(n, HEADLINE))
+    roofline = roofline_of(per_kernel, head_bytes, hbm, peak_src, lambda n: measured_traffic(n, HEADLINE),
+                           calls=2 * a.steps)
     if roofline:
-        roofline["units_per_launch"] = f"{w.batch * L1} tokens x {w.nheads} heads (one 16384-token call)"
+        roofline["units_per_call"] = f"{w.batch * L1} tokens x {w.nheads} heads (one 16384-token call)"
 
     # ---------------- end to end: pinned host inputs, copies inside the timed region
     e2e = None
@@ -704,7 +710,7 @@ def main():
             sms, sl = timed(scall, max(a.steps, 20), max(3, a.warmup))
             pk = profiled(lib, scall, max(a.steps, 20))
             rf = roofline_of(pk, lambda n, ww=wsub: kernel_bytes(n, ww, ww.batch, ww.seqlen, init), hbm, peak_src,
-                             lambda n, nm=name: measured_traffic(n, nm))
+                             lambda n, nm=name: measured_traffic(n, nm), calls=max(a.steps, 20))
             subs[name] = {
                 "workload": f"{name}: prefill b{wsub.batch} L{wsub.seqlen} H{wsub.nheads}xP{wsub.headdim} "
                             f"G{wsub.ngroups} N{wsub.dstate} Q{wsub.chunk} {wsub.act}"

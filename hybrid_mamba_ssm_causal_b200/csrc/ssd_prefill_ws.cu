@@ -43,6 +43,8 @@
 //                          epilogue of block k.
 // Variants: packed variable-length sequences on state slots (a CTA reads its sequence's
 // rows, length and slot from device arrays), and STATE_ONLY (final states and decay only).
+// Rows of fixed length may run as pieces over a series of launches (WsPieces), when whole rows
+// would leave the last wave of CTAs part-empty.
 // Hand-offs use mbarriers (all waits bounded):
 //   barCB  C'B'^T of a block done     bar0  C'H^T and B'^T(x'w) done     bar1  M x' done
 //   (tensor-core commits)
@@ -50,8 +52,9 @@
 //   barP   producer: block k's x', x'w and cumsum are in shared memory (3 slots: the producer
 //          may arrive for blocks k+1 and k+2 before a slow consumer waits for k)
 //   barM   consumer (one arrival per warp): C'B'^T of block k read, M of block k in TMEM
-//   barH   consumer (one arrival per warp): S^T of block k read, H^T of block k+1 written to
-//          shared memory, so the MMAs of block k+1 may start
+//   barH   consumer (one arrival per warp): phase 0, H^T of block 0 written; phase k+1, S^T of
+//          block k read and H^T of block k+1 written to shared memory, so the MMAs of block
+//          k+1 may start
 //   barE2  consumer: a block's x' and cumsum slots are free again (3 slots: x' and the cumsum
 //          live until the epilogue, so they rotate through three buffers)
 //   barW   the MMAs of a block are done, so its x'w slot is free again (2 slots: x'w is read
@@ -67,6 +70,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <type_traits>
 
@@ -282,10 +287,21 @@ struct WsMaps {
     CUtensorMap x, y, z;
 };
 
+// Rows split into pieces (runs of whole blocks), run as a series of launches: launch `round`
+// takes positions round * per_round ... of the queue [piece 0 of every (sequence, cluster),
+// piece 1 of every one, ...]. A piece's predecessor sits one queue length (the number of
+// (sequence, cluster) pairs, at least per_round) earlier, so it ran in an earlier launch; it
+// left the state in final_ssm, which the piece continues from. npieces = 1: one launch, one
+// whole row per cluster.
+struct WsPieces {
+    int round, per_round, npieces, piece_blocks;
+};
+
 // STATE_ONLY: the state-only pass (final states and decay of a prefill, no output rows): the
 // conv of x, B'^T(x'w) and the state recurrence.
 template <int R, bool SPLIT, bool STATE_ONLY>
-__global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillParams p, const __grid_constant__ WsMaps maps)
+__global__ void __launch_bounds__(kThreads, 1)
+    ssd_prefill_ws_kernel(PrefillParams p, const __grid_constant__ WsMaps maps, WsPieces pc)
 {
     using Lo = WsLayout<R>;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -294,7 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const int q = (int)cluster.block_rank();
     const int rpg = p.H / p.G;
     const int ncl = rpg / R;
-    const int64_t cid = blockIdx.x / R;
+    // this cluster's (sequence, head group) and, for a row split into pieces, the first block
+    // of its piece (pieces only for fixed-length rows, in the one-CTA full pass)
+    int64_t cid = blockIdx.x / R, k0 = 0;
+    if constexpr (R == 1 && !STATE_ONLY) {
+        if (pc.npieces > 1) {
+            const int64_t jobs = p.b * p.G * ncl;
+            const int64_t pos = (int64_t)pc.round * pc.per_round + cid;
+            cid = pos % jobs;
+            k0 = (pos / jobs) * pc.piece_blocks;
+        }
+    }
     const int64_t bi = cid / ((int64_t)p.G * ncl);
     const int g = (int)((cid / ncl) % p.G);
     const int h = g * rpg + (int)(cid % ncl) * R + q;
@@ -303,13 +329,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     // this CTA's sequence: its first token row, length, state slot, and whether it starts from
     // the states given (packed variable-length calls read them from their slot arrays)
     const bool varlen = p.cu_seqlens != nullptr;
-    const int64_t row0 = varlen ? (int64_t)p.cu_seqlens[bi] : bi * p.L;
-    const int64_t seqlen = varlen ? (int64_t)p.cu_seqlens[bi + 1] - row0 : p.L;
+    const int64_t row0 = varlen ? (int64_t)p.cu_seqlens[bi] : bi * p.L + k0 * kT;
+    const int64_t seqlen = varlen ? (int64_t)p.cu_seqlens[bi + 1] - row0
+                                  : min(p.L - k0 * kT, pc.npieces > 1 ? (int64_t)pc.piece_blocks * kT : p.L);
+    // a piece after the row's first continues from the state its predecessor left in final_ssm,
+    // and its conv halo is the row's own preceding tokens
+    const bool piece_cont = k0 > 0;
     const int64_t sidx = varlen && p.slot_idx ? (int64_t)p.slot_idx[bi] : bi;
     const bool cont = varlen ? (!p.has_init || p.has_init[bi] != 0) : true;
-    const bool init_ssm = cont && p.init_ssm != nullptr, init_conv = cont && p.init_conv != nullptr;
+    const bool init_ssm = piece_cont || (cont && p.init_ssm != nullptr);
+    const bool init_conv = !piece_cont && cont && p.init_conv != nullptr;
     // coordinates of token 0 in the tensor maps (token, sequence)
-    const int tmap_t0 = varlen ? (int)row0 : 0, tmap_b = varlen ? 0 : (int)bi;
+    const int tmap_t0 = varlen ? (int)row0 : (int)(k0 * kT), tmap_b = varlen ? 0 : (int)bi;
 
     float* mf = reinterpret_cast<float*>(smem + Lo::OFF_MISC);
     float* s_lam = mf + Lo::F_LAM;
@@ -365,8 +396,26 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     const bool consumer = tid >= kCons;
     const int crow = tid & 127, chalf = (tid - kCons) >> 7;   // consumer row and column half
     float H[32];
-    if (consumer) {
-        const float* h0 = init_ssm ? p.init_ssm + (sidx * p.H + h) * (int64_t)kP * kN : nullptr;
+    fence_before_sync();
+    __syncthreads();
+    cluster.sync();   // every peer's barriers are initialised before any remote arrival
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const float A2 = p.A[h] * 1.4426950408889634f;
+    const float Dh = STATE_ONLY ? 0.0f : p.D[h];
+    const float bias = p.dt_bias[h];
+    bool ok = true;
+    // a launch of a series of pieces lets the next launch start on the SMs its CTAs free; that
+    // launch waits for this one (griddepcontrol.wait) only where it reads what this one wrote
+    if (pc.npieces > 1 && tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // consumer: the state entering the first block (fp32 in registers, thread (n = row, half)
+    // keeps H^T[n][half*32 .. half*32+32)) and its bf16 copy for C'H^T; then the per-warp
+    // arrival on barH that lets block 0's products start. A continuing piece first waits for the
+    // earlier launches, whose last one wrote the state it continues from.
+    auto init_state = [&]() {
+        if (piece_cont) asm volatile("griddepcontrol.wait;" ::: "memory");
+        const float* h0 = init_ssm ? (piece_cont ? p.final_ssm : p.init_ssm) + (sidx * p.H + h) * (int64_t)kP * kN : nullptr;
 #pragma unroll
         for (int i = 0; i < 32; ++i) H[i] = h0 ? h0[(int64_t)(chalf * 32 + i) * kN + crow] : 0.0f;
         unsigned char* sH = smem + Lo::OFF_H;
@@ -378,16 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             *reinterpret_cast<uint4*>(sH + canon_off(crow, chalf * 32 + 8 * v, kP)) = u;
         }
         fence_async_smem();
-    }
-    fence_before_sync();
-    __syncthreads();
-    cluster.sync();   // every peer's barriers are initialised before any remote arrival
-    fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
-    const float A2 = p.A[h] * 1.4426950408889634f;
-    const float Dh = STATE_ONLY ? 0.0f : p.D[h];
-    const float bias = p.dt_bias[h];
-    bool ok = true;
+        fence_before_sync();
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive_local(barH);
+    };
 
     const int64_t nblk = (seqlen + kT - 1) / kT;
     auto blen = [&](int64_t k) { return (int)min((int64_t)kT, seqlen - k * kT); };
@@ -563,10 +606,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
             if (tid == 32 && m + XBUF < nblk) load_x(m + XBUF);   // its stage has been read
             if (tid == 0) mbar_arrive_local(barP + 8 * s3(m));
         }
-        // final conv state of the head's x channels: the last three raw inputs
+        // final conv state of the head's x channels: the last three raw inputs. Of a row run as
+        // pieces only the last piece writes it, and only once the earlier launches are done: a
+        // short piece's producer can finish before them, and a first piece may still have to read
+        // the initial conv state that the final one overwrites in place.
         const int len_last = nblk > 0 ? blen(nblk - 1) : 0;
+        const bool row_end = pc.npieces == 1 || k0 * kT + seqlen >= p.L;
+        if (pc.npieces > 1 && row_end) asm volatile("griddepcontrol.wait;" ::: "memory");
         named_sync(kBarProd, kProd);
-        for (int e = tid; e < 3 * kP; e += kProd) {
+        for (int e = tid; e < 3 * kP && row_end; e += kProd) {
             const int kk = e / kP, c = e % kP;
             const uint4* stl = stage + (nblk > 0 ? ((nblk - 1) % XBUF) * kStageU4 : 0);
             const __nv_bfloat16 v =
@@ -578,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         // has read the initial state before this kernel started, and each thread reads its
         // channel's three values before writing them, so the final state may share memory with
         // the initial one.
-        if (h == g * rpg) {
+        if (h == g * rpg && row_end) {
             for (int c = tid; c < 2 * kN; c += kProd) {
                 const bool isC = c >= kN;
                 const int64_t ch = (isC ? GN : 0) + (int64_t)g * kN + (c % kN);   // within [B | C]
@@ -589,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
 #pragma unroll
                 for (int kk = 0; kk < 3; ++kk) {
                     const int64_t idx = seqlen + kk;   // into [initial state (3) ; tokens]
-                    if (idx < 3) v3[kk] = init_conv ? ic[idx] : __float2bfloat16_rn(0.0f);
+                    if (idx < 3 && !piece_cont) v3[kk] = init_conv ? ic[idx] : __float2bfloat16_rn(0.0f);
                     else v3[kk] = src[(row0 + idx - 3) * ld];
                 }
                 __nv_bfloat16* fc = (__nv_bfloat16*)p.final_conv + (sidx * Cc + HP + ch) * 3;
@@ -649,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
                 // this block's x'w (barP); the consumer has read S^T of block k-1 and written H^T
                 // for this block (barH)
                 if (ok && !mbar_wait_bounded(barP + 8 * s3(k), p3(k), kWaitLimit)) ok = false;
-                if (k >= 1 && ok && !mbar_wait_bounded(barH, (uint32_t)((k - 1) & 1), kWaitLimit)) ok = false;
+                if (ok && !mbar_wait_bounded(barH, (uint32_t)(k & 1), kWaitLimit)) ok = false;
                 fence_after_sync();
                 const uint32_t colYs = kColYs0 + 64 * (uint32_t)sl;
                 const uint32_t aXWs = aXW + 16384 * (uint32_t)sl;
@@ -676,6 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         }
     } else if constexpr (STATE_ONLY) {
         // ================= consumer of the state-only pass (warps 8..15) =================
+        init_state();
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         float lam_tot = 0.0f;   // sum of delta*A over the row, log2 units
         for (int64_t k = 0; k < nblk; ++k) {
@@ -706,6 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
         if (tid == kCons && p.decay) p.decay[bi * p.H + h] = ex2(lam_tot);
     } else {
         // =========================== consumer (warps 8..15) ===========================
+        init_state();
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t aY = s_base + Lo::OFF_Y;
         // byte offset of 16-byte chunk c of token row r in the swizzled y tile
@@ -964,6 +1014,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_prefill_ws_kernel(PrefillPara
     }
 
     if (!ok) set_device_status(p.status, kDevTimeout);
+    // a launch of pieces completes only after the launch before it, so a piece whose predecessor
+    // ran several launches back still finds its state written
+    if (pc.npieces > 1 && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     fence_before_sync();
     __syncthreads();
     cluster.sync();   // no peer still arrives on this CTA's shared memory
@@ -1080,6 +1133,44 @@ cudaError_t launch_bc_conv(const PrefillParams& p, int nch, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// Pieces per row for `jobs` rows of `nblk` blocks, one CTA per SM on `sms` SMs: whole rows
+// leave the last wave part-empty (256 rows on 148 SMs run as two waves, the second 108 wide).
+// The plan minimises launches x (blocks per piece + about 1.5 blocks for the fill and drain of
+// a launch's pipelines); with fewer rows than SMs it keeps rows whole. The environment
+// variable SSD_MIXER_PREFILL_PIECES (read once; 1 .. 64) fixes the number of pieces instead.
+WsPieces plan_pieces(int64_t jobs, int64_t nblk, int sms)
+{
+    static const int forced = [] {
+        const char* v = getenv("SSD_MIXER_PREFILL_PIECES");
+        const int n = v ? atoi(v) : 0;
+        return n >= 1 && n <= 64 ? n : 0;
+    }();
+    const WsPieces whole{0, (int)jobs, 1, (int)nblk};   // one launch, every row whole
+    if (nblk < 2 || (!forced && jobs < sms)) return whole;
+    WsPieces pc{0, (int)std::min((int64_t)sms, jobs), 1, (int)nblk};
+    double best = 0.0;
+    for (int n = forced ? forced : 1; n <= (forced ? forced : 8) && n <= nblk; ++n) {
+        const int64_t pb = (nblk + n - 1) / n, np = (nblk + pb - 1) / pb;
+        const int64_t launches = (jobs * np + sms - 1) / sms;
+        const double cost = (double)launches * ((double)pb + 1.5);
+        if (n == (forced ? forced : 1) || cost < best) {
+            best = cost;
+            pc.npieces = (int)np;
+            pc.piece_blocks = (int)pb;
+        }
+    }
+    return pc.npieces > 1 ? pc : whole;
+}
+
+int sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+        return 148;
+    return sms;
+}
+
 template <int R, bool SPLIT, bool STATE_ONLY = false>
 cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
 {
@@ -1104,17 +1195,29 @@ cudaError_t launch_ws(const PrefillParams& p, cudaStream_t st)
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = Lo::TOTAL;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = R;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    // one CTA per SM (R = 1, no cluster): rows of fixed length may run as pieces, each launch
+    // after the first allowed to start while the one before it finishes
+    const int64_t jobs = p.b * p.H / R;
+    WsPieces pc{0, (int)jobs, 1, 0};
+    if (R == 1 && !STATE_ONLY && !p.cu_seqlens) pc = plan_pieces(jobs, (p.L + kT - 1) / kT, sm_count());
+    const int64_t total = jobs * pc.npieces;
     {
-        LaunchScope ls(STATE_ONLY ? "tc_prefill_state" : "tc_prefill", st);
-        e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT, STATE_ONLY>, p, maps);
-        if (e != cudaSuccess) return e;
+        LaunchScope ls(STATE_ONLY ? "tc_prefill_state" : "tc_prefill", st, (int)((total + pc.per_round - 1) / pc.per_round));
+        for (pc.round = 0; (int64_t)pc.round * pc.per_round < total; ++pc.round) {
+            cfg.gridDim = dim3((unsigned)(R * std::min((int64_t)pc.per_round, total - (int64_t)pc.round * pc.per_round)));
+            cfg.numAttrs = pc.round > 0 ? 2 : 1;
+            e = cudaLaunchKernelEx(&cfg, ssd_prefill_ws_kernel<R, SPLIT, STATE_ONLY>, p, maps, pc);
+            if (e != cudaSuccess) return e;
+        }
     }
     if (SPLIT && !STATE_ONLY && p.rows() > 0 && !p.defer_norm) {
         LaunchScope ls("tc_norm_finish", st);

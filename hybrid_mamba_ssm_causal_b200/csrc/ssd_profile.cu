@@ -14,6 +14,7 @@ namespace {
 struct Rec {
     const char* name;
     cudaEvent_t a, b;
+    int launches;
 };
 
 std::atomic<long long> g_launches{0};
@@ -23,12 +24,12 @@ std::vector<Rec> g_recs;
 
 }  // namespace
 
-void profile_begin(const char* name, cudaStream_t st, void** token)
+void profile_begin(const char* name, cudaStream_t st, void** token, int launches)
 {
-    g_launches.fetch_add(1, std::memory_order_relaxed);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
     *token = nullptr;
     if (!g_enabled.load(std::memory_order_relaxed)) return;
-    Rec* r = new Rec{name, nullptr, nullptr};
+    Rec* r = new Rec{name, nullptr, nullptr, launches};
     if (cudaEventCreate(&r->a) != cudaSuccess) {
         delete r;
         return;
@@ -84,7 +85,7 @@ int ssd_mixer_profile_read(const char** names, double* total_ms, int* launches, 
             ++n;
         }
         if (timed) total_ms[k] += ms;   // a pair that could not be timed still counts as a launch
-        launches[k] += 1;
+        launches[k] += r.launches;
     }
     return n;
 }

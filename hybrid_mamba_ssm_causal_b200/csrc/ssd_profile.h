@@ -10,13 +10,15 @@
 
 namespace ssd {
 
-void profile_begin(const char* name, cudaStream_t st, void** token);
+void profile_begin(const char* name, cudaStream_t st, void** token, int launches);
 void profile_end(void* token, cudaStream_t st);
 
+// `launches`: the kernel launches the scope encloses (a series of launches that may overlap,
+// such as the pieces of one prefill call, is timed as one span with no events between them).
 struct LaunchScope {
     void* token = nullptr;
     cudaStream_t st;
-    LaunchScope(const char* name, cudaStream_t s) : st(s) { profile_begin(name, s, &token); }
+    LaunchScope(const char* name, cudaStream_t s, int launches = 1) : st(s) { profile_begin(name, s, &token, launches); }
     ~LaunchScope() { profile_end(token, st); }
 };
 

@@ -436,8 +436,9 @@ SSD_API long long ssd_mixer_launch_count(void);
 
 /* Switch per-kernel timing on (1) or off (0). While on, every kernel launch is
  * bracketed by a pair of CUDA events recorded on the launching stream (a few
- * microseconds of host overhead per launch; the kernels themselves are unchanged).
- * Off by default. */
+ * microseconds of host overhead per launch; the kernels themselves are unchanged). The
+ * launches of one prefill call whose rows run as pieces may overlap one another, so they
+ * share one pair: one span, counted as that many launches. Off by default. */
 SSD_API void ssd_mixer_profile_enable(int on);
 
 /* Collects the event pairs recorded since the last read: waits for each to complete

@@ -20,7 +20,7 @@ def test_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "KERNEL_SOURCES", {"kern": ["k/kern.cu"]})
     h = bench.sources_sha256("kern")
     (tmp_path / bench.TRAFFIC_FILE).write_text(json.dumps({"entries": [
-        {"kernel": "kern", "workload": "wl", "traffic_bytes_per_launch": 12345, "kernel_sources_sha256": h}]}))
+        {"kernel": "kern", "workload": "wl", "traffic_bytes_per_call": 12345, "kernel_sources_sha256": h}]}))
     assert bench.measured_traffic("kern", "wl") == 12345.0
     # another workload has no figure
     assert bench.measured_traffic("kern", "other_wl") is None
@@ -42,5 +42,5 @@ def test_committed_traffic_file_is_well_formed():
     data = json.load(open(path))
     for e in data["entries"]:
         assert e["kernel"] in bench.KERNEL_SOURCES
-        assert float(e["traffic_bytes_per_launch"]) > 0
+        assert float(e["traffic_bytes_per_call"]) > 0
         assert len(e["kernel_sources_sha256"]) == 64 and e["workload"] and e["command"]
