@@ -212,6 +212,20 @@ int ssd_mixer_prefill_path(const ssd_dims* d)
                                                                                            : SSD_PATH_CUDA_CORES;
 }
 
+ssd_status ssd_mixer_prefill_plan(const ssd_dims* d, int sms, int* launches, int* pieces, int* piece_blocks,
+                                  int* ctas_per_launch)
+{
+    if (ssd_mixer_prefill_path(d) != SSD_PATH_TENSOR_CORES) return SSD_ERR_UNSUPPORTED;
+    if (!launches || !pieces || !piece_blocks || !ctas_per_launch || sms < 0) return SSD_ERR_INVALID_ARG;
+    const ssd::PrefillPlan pl =
+        ssd::prefill_ws_plan(d->batch, d->seqlen, d->nheads, d->ngroups, sms > 0 ? sms : ssd::device_sm_count());
+    *launches = d->batch > 0 && d->seqlen > 0 ? pl.launches : 0;
+    *pieces = pl.pieces;
+    *piece_blocks = pl.piece_blocks;
+    *ctas_per_launch = pl.ctas_per_launch;
+    return SSD_OK;
+}
+
 ssd_status ssd_mixer_prefill_stage_offsets(const ssd_dims* d, size_t* xbc_act, size_t* delta, size_t* y_pre)
 {
     if (ssd_mixer_prefill_path(d) != SSD_PATH_CUDA_CORES) return SSD_ERR_UNSUPPORTED;

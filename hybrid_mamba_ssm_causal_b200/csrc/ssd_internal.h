@@ -174,6 +174,14 @@ cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int
 // The state-only pass on the tensor-core path: final states and decay, no output rows.
 cudaError_t launch_prefill_state_ws(const PrefillParams& p, cudaStream_t stream);
 cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream);
+// How the tensor-core main kernel runs a fixed-length call of b rows of L tokens on `sms` SMs:
+// launches per call, pieces per (sequence, head) row, 128-token blocks per piece (the last
+// piece of a row may be shorter), CTAs per launch (the last launch may have fewer).
+struct PrefillPlan {
+    int launches, pieces, piece_blocks, ctas_per_launch;
+};
+PrefillPlan prefill_ws_plan(int64_t b, int64_t L, int H, int G, int sms);
+int device_sm_count();
 // The tensor-core path keeps SiLU(conv) of B and C in the workspace as 32 KB chunks, one per
 // (128-token block of a sequence, matrix B or C, group): chunk ((s + floor(start_s / 128) + k) * 2
 // + matrix) * G + group holds block k of sequence s (first packed row start_s) in the MMA operand

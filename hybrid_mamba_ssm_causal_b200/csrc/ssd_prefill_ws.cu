@@ -1237,6 +1237,18 @@ cudaError_t launch_prefill_state_ws(const PrefillParams& p, cudaStream_t stream)
     return launch_ws<1, false, true>(p, stream);
 }
 
+PrefillPlan prefill_ws_plan(int64_t b, int64_t L, int H, int G, int sms)
+{
+    const int r = H / G, R = (r == 2 || r == 4) ? r : 1;
+    const int64_t jobs = b * H / R, nblk = (L + kT - 1) / kT;
+    const WsPieces pc = R == 1 ? plan_pieces(jobs, nblk, sms) : WsPieces{0, (int)jobs, 1, (int)nblk};
+    const int64_t total = jobs * pc.npieces;
+    return PrefillPlan{(int)((total + pc.per_round - 1) / std::max(1, pc.per_round)), pc.npieces, pc.piece_blocks,
+                       pc.per_round * R};
+}
+
+int device_sm_count() { return sm_count(); }
+
 // Groups of 2 or 4 heads: one cluster per group, the norm fused; wider groups: no cluster,
 // the norm finished by ws_norm_finish_kernel.
 cudaError_t launch_prefill_ws(const PrefillParams& p, cudaStream_t stream)

@@ -39,7 +39,8 @@ SYMBOLS = ("ssd_mixer_prefill_workspace_size", "ssd_mixer_prefill", "ssd_mixer_d
            "ssd_mixer_prefill_static", "ssd_mixer_prefill_varlen_workspace_size", "ssd_mixer_prefill_varlen",
            "ssd_mixer_prefill_state_workspace_size", "ssd_mixer_prefill_state", "ssd_mixer_state_pass",
            "ssd_mixer_backward_workspace_size", "ssd_mixer_backward", "ssd_mixer_selftest_wait",
-           "ssd_mixer_prefill_static_status", "ssd_mixer_prefill_path", "ssd_mixer_prefill_stage_offsets",
+           "ssd_mixer_prefill_static_status", "ssd_mixer_prefill_path", "ssd_mixer_prefill_plan",
+           "ssd_mixer_prefill_stage_offsets",
            "ssd_mixer_projection", "ssd_mixer_layer_workspace_size", "ssd_mixer_layer_prefill")
 SSD_PATH_NONE, SSD_PATH_CUDA_CORES, SSD_PATH_TENSOR_CORES = range(3)
 
@@ -124,6 +125,9 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_mixer_layer_prefill.restype = ctypes.c_int
     lib.ssd_mixer_prefill_path.argtypes = [ctypes.POINTER(_CDims)]
     lib.ssd_mixer_prefill_path.restype = ctypes.c_int
+    IP = ctypes.POINTER(ctypes.c_int)
+    lib.ssd_mixer_prefill_plan.argtypes = [ctypes.POINTER(_CDims), ctypes.c_int, IP, IP, IP, IP]
+    lib.ssd_mixer_prefill_plan.restype = ctypes.c_int
     SZP = ctypes.POINTER(ctypes.c_size_t)
     lib.ssd_mixer_prefill_stage_offsets.argtypes = [ctypes.POINTER(_CDims), SZP, SZP, SZP]
     lib.ssd_mixer_prefill_stage_offsets.restype = ctypes.c_int
@@ -312,6 +316,17 @@ def ssd_mixer_prefill_path(dims: Dims) -> int:
     these dims runs (a host-side query)."""
     cd = dims.c()
     return int(load_library().ssd_mixer_prefill_path(ctypes.byref(cd)))
+
+
+def ssd_mixer_prefill_plan(dims: Dims, sms: int = 0) -> dict:
+    """How the tensor-core main kernel runs a prefill of these dims on ``sms`` SMs (0 = this
+    device's): launches per call, pieces per (sequence, head) row, blocks per piece, CTAs per
+    launch (a host-side query)."""
+    cd = dims.c()
+    out = [ctypes.c_int(0) for _ in range(4)]
+    st = load_library().ssd_mixer_prefill_plan(ctypes.byref(cd), sms, *[ctypes.byref(o) for o in out])
+    _check(st, "ssd_mixer_prefill_plan")
+    return dict(zip(("launches", "pieces", "piece_blocks", "ctas_per_launch"), (o.value for o in out)))
 
 
 def prefill_uses_tensor_cores(dims: Dims) -> bool:

@@ -141,6 +141,21 @@ typedef enum ssd_path {
 } ssd_path;
 SSD_API int ssd_mixer_prefill_path(const ssd_dims* dims);
 
+/* How ssd_mixer_prefill runs the tensor-core main kernel for `dims` (a host-side query;
+ * nothing is launched; no counterpart in the pages). Each (sequence, head) row is a walk over
+ * its 128-token blocks, one CTA per SM. When the rows of a group wider than a cluster outnumber
+ * the SMs, whole rows would leave the last wave of CTAs part-empty. The call then splits every
+ * row into pieces of whole blocks and runs them as a series of launches. Each piece continues
+ * from the state its predecessor left in final_ssm_state, written by an earlier launch.
+ * sms: the SM count to plan for, 0 = the current device's (148 when none can be queried).
+ * Writes the launches per call (0 for an empty call), the pieces per row, the blocks per piece
+ * (the last piece of a row may be shorter) and the CTAs per launch (the last launch may have
+ * fewer). The environment variable SSD_MIXER_PREFILL_PIECES (read once per process, 1 .. 64)
+ * fixes the piece count. Returns SSD_ERR_UNSUPPORTED unless the dims take the tensor-core path
+ * (ssd_mixer_prefill_path), SSD_ERR_INVALID_ARG for a NULL output or a negative sms. */
+SSD_API ssd_status ssd_mixer_prefill_plan(const ssd_dims* dims, int sms, int* launches, int* pieces,
+                                          int* piece_blocks, int* ctas_per_launch);
+
 /* Where a CUDA-core prefill (SSD_PATH_CUDA_CORES) leaves its intermediates in its workspace,
  * for checking each stage on its own: byte offsets from the workspace start of
  *   xbc_act [b][L][Cc] activation dtype: SiLU(conv) of [x|B|C];

@@ -231,3 +231,48 @@ def test_layer_and_projection_refuse_unsupported_arguments(lib):
     assert lib.ssd_mixer_projection(4, 8, 12, FAKE, 16, FAKE, 16, FAKE, 8, FAKE, None) == sm.SSD_ERR_UNSUPPORTED
     assert lib.ssd_mixer_projection(4, 8, 16, FAKE, 16, FAKE, 16, FAKE, 8, FAKE + 8, None) == sm.SSD_ERR_INVALID_ARG
     assert lib.ssd_mixer_projection(0, 8, 16, None, 16, None, 16, None, 8, FAKE, None) == sm.SSD_OK
+
+
+def _tc(b, L, H, G):
+    return _dims(batch=b, seqlen=L, nheads=H, ngroups=G, headdim=64, dstate=128)
+
+
+def test_prefill_plan_query(lib):
+    """The main kernel's launch plan (host logic, nothing launched): whole rows in one launch
+    unless rows of a group wider than a cluster outnumber the SMs; then pieces over a series of
+    launches in which every piece's predecessor ran in an earlier launch."""
+    if os.environ.get("SSD_MIXER_PREFILL_PIECES"):
+        pytest.skip("piece count fixed by the environment")
+    plan = lambda *a: sm.ssd_mixer_prefill_plan(_tc(*a), sms=148)
+    # long_bf16 call: 256 rows of 128 blocks -> 4 pieces of 32, 7 launches (224 block-times, not 256)
+    assert plan(1, 16384, 256, 8) == dict(launches=7, pieces=4, piece_blocks=32, ctas_per_launch=148)
+    # mid_bf16: 512 rows of 32 blocks -> 2 pieces of 16, 7 launches (112, not 128)
+    assert plan(8, 4096, 64, 8) == dict(launches=7, pieces=2, piece_blocks=16, ctas_per_launch=148)
+    # small_bf16: groups of 4 heads held by clusters of 4 -> one launch of whole rows
+    assert plan(2, 2048, 32, 8) == dict(launches=1, pieces=1, piece_blocks=16, ctas_per_launch=64)
+    # fewer rows than SMs, and 256 short rows that pieces would not help: one launch
+    assert plan(1, 16384, 64, 8) == dict(launches=1, pieces=1, piece_blocks=128, ctas_per_launch=64)
+    assert plan(2, 300, 128, 16) == dict(launches=1, pieces=1, piece_blocks=3, ctas_per_launch=256)
+    assert plan(0, 300, 128, 16)["launches"] == 0 and plan(2, 0, 128, 16)["launches"] == 0
+    # invariants over a sweep, checked by replaying the queue of pieces launch by launch
+    for b in (1, 2, 3, 5):
+        for H, G in ((64, 8), (128, 16), (256, 8), (96, 12)):
+            for L in (1, 129, 1000, 4096, 16384):
+                p = plan(b, L, H, G)
+                rows, nblk = b * H, -(-L // 128)
+                if p["pieces"] == 1:
+                    assert p["launches"] == 1 and p["ctas_per_launch"] == rows
+                    continue
+                per, pb, n = p["ctas_per_launch"], p["piece_blocks"], p["pieces"]
+                assert rows >= 148 and per <= rows
+                assert (n - 1) * pb < nblk <= n * pb
+                assert p["launches"] == -(-rows * n // per)
+                for pos in range(rows, rows * n):              # a piece after the first of its row
+                    assert (pos - rows) // per < pos // per    # its predecessor ran in an earlier launch
+    # other SM counts plan for their own waves
+    assert sm.ssd_mixer_prefill_plan(_tc(1, 16384, 256, 8), sms=256)["pieces"] == 1
+    # only the tensor-core path has a plan
+    with pytest.raises(sm.SsdError):
+        sm.ssd_mixer_prefill_plan(_dims(act="f32", headdim=64, dstate=128), sms=148)
+    with pytest.raises(sm.SsdError):
+        sm.ssd_mixer_prefill_plan(_tc(1, 16384, 256, 8), sms=-1)
