@@ -28,6 +28,8 @@ cases = [
     base.with_(batch=2, seqlen=513, nheads=16, ngroups=2, init_ssm_std=0.1, init_conv_std=1.0, seed=21),
     # 130 tokens: a second piece of 2 tokens, shorter than the conv window
     base.with_(batch=3, seqlen=130, nheads=8, ngroups=1, init_ssm_std=0.0, init_conv_std=0.0, seed=22),
+    # 512 tokens = 4 whole blocks: 2 or 4 pieces of equal length
+    base.with_(batch=2, seqlen=512, nheads=16, ngroups=2, init_ssm_std=0.1, init_conv_std=1.0, seed=25),
 ]
 for w in cases:
     inp = make_prefill_inputs(w)
@@ -73,10 +75,10 @@ def run_with_pieces(n: int, library: str | None = None):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("n", [2, 3, 5])
+@pytest.mark.parametrize("n", [2, 3, 4, 5])
 def test_rows_in_pieces_match_the_oracle(n):
-    """n = 2: pieces of 3 and 2 blocks; 3: the last piece is the one-token block; 5: every
-    block its own piece."""
+    """On 513 tokens, n = 2: pieces of 3 and 2 blocks; 3: the last piece is the one-token block;
+    5: every block its own piece. On 512 tokens, 2 and 4 pieces are equally long."""
     run_with_pieces(n)
 
 
